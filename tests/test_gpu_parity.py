@@ -1,0 +1,347 @@
+"""GPU path vs the CPU oracle, through the C ABI (tiny and small shapes).
+
+Tolerances: plan bit-exact when fed the oracle's float32 pi; scores within
+1e-3 relative (entries >= 1e-6 of the row max; smaller ones 1e-9 absolute);
+pi from the GPU water-fill within 1e-5 relative; forward within max-abs 2e-2
+and relative-L2 5e-3 of the oracle on the same plan (bf16 inputs, fp32
+accumulation).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_sparse_attention_12_b200 import abi, inputs
+
+pytestmark = pytest.mark.gpu
+
+W = inputs.TINY
+SCALE = 1 / math.sqrt(W.d)
+
+
+def cfg_of(w, **kw):
+    c = abi.Config(kv_block=w.kv_block, budget=w.budget, n_clusters=w.n_clusters,
+                   kmeans_iters=w.kmeans_iters, seed=w.seed)
+    for k, v in kw.items():
+        setattr(c, k, v)
+    return c
+
+
+def assert_forward_close(Og, Oo, what=""):
+    Og = np.asarray(Og, dtype=np.float64)
+    err = np.abs(Og - Oo).max()
+    rel = np.linalg.norm(Og - Oo) / max(np.linalg.norm(Oo), 1e-30)
+    assert err <= 2e-2 and rel <= 5e-3, f"{what}: max-abs {err:.3e}, rel-L2 {rel:.3e}"
+    return err, rel
+
+
+def assert_scores_close(Sg, So):
+    Sg = np.asarray(Sg, dtype=np.float64)
+    mx = So.max(axis=-1, keepdims=True)
+    big = So >= 1e-6 * mx
+    rel = np.abs(Sg - So) / np.maximum(So, 1e-300)
+    assert rel[big].max() <= 1e-3, rel[big].max()
+    assert np.abs(Sg - So)[~big].max(initial=0) <= 1e-9
+
+
+@pytest.fixture(scope="module")
+def tiny():
+    Qc, Kc, Vc = inputs.make_qkv(W)
+    sel = oracle.selector_all(Qc, Kc, 128, W.kv_block, W.n_clusters, W.kmeans_iters, SCALE)
+    return dict(Qc=Qc, Kc=Kc, Vc=Vc, Q=Qc.cuda(), K=Kc.cuda(), V=Vc.cuda(), sel=sel)
+
+
+# ------------------------------------------------------------------ selector
+
+def test_library_loads_and_reports_version():
+    assert "sm_100a" in abi.version()
+
+
+def test_meanpool_parity(tiny):
+    Kb = abi.meanpool(tiny["K"], W.kv_block)
+    abi.check()
+    np.testing.assert_allclose(Kb.cpu().numpy(), tiny["sel"]["Kbar"], rtol=1e-6, atol=1e-6)
+
+
+@pytest.mark.parametrize("kb,N", [(128, 300), (8, 4096), (4, 1000)])
+def test_meanpool_ragged(kb, N):
+    K = torch.randn(1, 3, N, 64, generator=torch.Generator().manual_seed(N)).to(torch.bfloat16)
+    Kb = abi.meanpool(K.cuda(), kb)
+    abi.check()
+    for h in range(3):
+        np.testing.assert_allclose(Kb[0, h].cpu().numpy(), oracle.meanpool(K[0, h], kb), rtol=1e-6, atol=1e-6)
+
+
+def test_kmeans_parity(tiny):
+    cfg = cfg_of(W)
+    C, w, lab = abi.kmeans(tiny["Q"], cfg)
+    abi.check()
+    C, w, lab = C.cpu().numpy(), w.cpu().numpy(), lab.cpu().numpy()
+    So = tiny["sel"]
+    agree_rows, agree_lab = 0, 0
+    nrows = lab.shape[2] * lab.shape[1]
+    for h in range(W.H):
+        for qb in range(lab.shape[2]):
+            lo = So["labels"][0, h, qb]
+            lg = lab[0, h, qb]
+            agree_lab += (lo == lg).sum()
+            if np.array_equal(lo, lg):
+                agree_rows += 1
+                np.testing.assert_allclose(C[0, h, qb], So["C"][0, h, qb], rtol=1e-5, atol=1e-5)
+                np.testing.assert_array_equal(w[0, h, qb], So["w"][0, h, qb].astype(np.float32))
+    print(f"k-means: {agree_rows}/{nrows} rows identical, label agreement {agree_lab / (nrows * 128):.5f}")
+    assert agree_lab / (nrows * 128) >= 0.99
+    assert agree_rows >= 0.9 * nrows
+
+
+def test_kmeans_ragged_block_and_few_clusters():
+    N, d = 1000, 128
+    Q = torch.randn(1, 2, N, d, generator=torch.Generator().manual_seed(5)).to(torch.bfloat16)
+    cfg = abi.Config(n_clusters=5, kmeans_iters=7)
+    C, w, lab = abi.kmeans(Q.cuda(), cfg)
+    abi.check()
+    qb = N // 128  # ragged block, 104 rows
+    Co, wo, lo = oracle.kmeans(Q[0, 1, qb * 128:], 5, 7)
+    lg = lab[0, 1, qb].cpu().numpy()
+    assert np.all(lg[N - qb * 128:] == -1)
+    np.testing.assert_array_equal(lg[:N - qb * 128], lo)
+    np.testing.assert_allclose(C[0, 1, qb].cpu().numpy(), Co, rtol=1e-5, atol=1e-5)
+    np.testing.assert_array_equal(w[0, 1, qb].cpu().numpy(), wo.astype(np.float32))
+
+
+def test_score_parity_fed_inputs(tiny):
+    """Scores from the oracle's own centroids, weights and mean keys (rounded
+    to float32, the kernel's input type), against the oracle on the same
+    rounded inputs."""
+    So = tiny["sel"]
+    C32 = torch.from_numpy(So["C"]).float()
+    w32 = torch.from_numpy(So["w"]).float()
+    K32 = torch.from_numpy(So["Kbar"]).float()
+    Sg = abi.score(C32.cuda(), w32.cuda(), K32.cuda(), tuple(tiny["Q"].shape), cfg_of(W))
+    abi.check()
+    Sg = Sg.cpu().numpy()
+    for h in range(W.H):
+        for qb in range(0, Sg.shape[2], 3):
+            so = oracle.scores(C32[0, h, qb].double(), w32[0, h, qb].double(), K32[0, h].double(), SCALE)
+            assert_scores_close(Sg[0, h, qb], so)
+            assert abs(Sg[0, h, qb].sum() - 1) < 1e-4
+
+
+def test_score_parity_end_to_end(tiny):
+    cfg = cfg_of(W)
+    shape = tuple(tiny["Q"].shape)
+    Kb = abi.meanpool(tiny["K"], W.kv_block)
+    C, w, lab = abi.kmeans(tiny["Q"], cfg)
+    Sg = abi.score(C, w, Kb, shape, cfg)
+    abi.check()
+    Sg, lab = Sg.cpu().numpy(), lab.cpu().numpy()
+    So = tiny["sel"]
+    checked = 0
+    for h in range(W.H):
+        for qb in range(Sg.shape[2]):
+            if np.array_equal(lab[0, h, qb], So["labels"][0, h, qb]):
+                assert_scores_close(Sg[0, h, qb], So["S"][0, h, qb])
+                checked += 1
+    assert checked >= 0.9 * W.H * Sg.shape[2]
+
+
+# ------------------------------------------------------------------ planner
+
+def test_plan_from_pi_bit_exact(tiny):
+    cfg = cfg_of(W)
+    shape = tuple(tiny["Q"].shape)
+    po = oracle.plan_all(tiny["sel"]["S"], W.budget, 0, W.seed, want_pi=True)
+    pi = torch.from_numpy(po["pi"])
+    pg = abi.plan_from_pi(pi.cuda(), shape, cfg)
+    abi.check()
+    assert pg.cap == po["cap"]
+    cg = pg.counts.cpu().numpy()
+    np.testing.assert_array_equal(cg, po["counts"])
+    ig, sg = pg.idx.cpu().numpy(), pg.pi_sel.cpu().numpy()
+    for r in np.ndindex(cg.shape):
+        n = cg[r]
+        np.testing.assert_array_equal(ig[r][:n], po["idx"][r][:n])
+        np.testing.assert_array_equal(sg[r][:n], po["pi_sel"][r][:n])
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2**40 + 7])
+def test_plan_from_pi_bit_exact_random_pi(seed):
+    B, H, N, d = 2, 3, 2000, 64
+    nqb, nkvb = -(-N // 128), N // 4
+    g = np.random.default_rng(seed % 1000)
+    pi = g.random((B, H, nqb, nkvb)).astype(np.float32) ** 3
+    pi[..., ::17] = 1.0
+    pi[..., 5::23] = 0.0
+    cfg = abi.Config(kv_block=4, budget=0.3, seed=seed)
+    pg = abi.plan_from_pi(torch.from_numpy(pi).cuda(), (B, H, N, d), cfg)
+    abi.check()
+    cg, ig, sg = pg.counts.cpu().numpy(), pg.idx.cpu().numpy(), pg.pi_sel.cpu().numpy()
+    for b in range(B):
+        for h in range(H):
+            for qb in range(nqb):
+                idx, ps, n = oracle.sample(pi[b, h, qb], seed, b, h, qb, pg.cap)
+                assert cg[b, h, qb] == min(n, pg.cap)
+                np.testing.assert_array_equal(ig[b, h, qb, :cg[b, h, qb]], idx)
+                np.testing.assert_array_equal(sg[b, h, qb, :cg[b, h, qb]], ps)
+
+
+def test_waterfill_pi_parity(tiny):
+    cfg = cfg_of(W)
+    shape = tuple(tiny["Q"].shape)
+    S32 = torch.from_numpy(tiny["sel"]["S"]).float()
+    pg, pig = abi.plan_from_scores(S32.cuda(), shape, cfg, want_pi=True)
+    abi.check()
+    pig = pig.cpu().numpy()
+    S64 = S32.double().numpy()
+    po = oracle.plan_all(S64, W.budget, 0, W.seed, want_pi=True)
+    rel = np.abs(pig - po["pi"]) / np.maximum(po["pi"], 1e-30)
+    assert rel.max() <= 1e-5
+    exact = np.mean(pig == po["pi"])
+    print(f"water-fill: {exact:.6f} of pi bit-identical, max rel {rel.max():.2e}")
+    # when every pi agrees bit for bit, so must the sampled plan
+    if exact == 1.0:
+        np.testing.assert_array_equal(pg.counts.cpu().numpy(), po["counts"])
+
+
+def test_topk_bit_exact_from_fp32_scores(tiny):
+    cfg = cfg_of(W, mode=abi.MODE_TOPK)
+    shape = tuple(tiny["Q"].shape)
+    S32 = torch.from_numpy(tiny["sel"]["S"]).float()
+    S32[0, 0, 0, 10:40] = S32[0, 0, 0, 10]  # ties across the threshold
+    pg = abi.plan_from_scores(S32.cuda(), shape, cfg)
+    abi.check()
+    po = oracle.plan_all(S32.double().numpy(), W.budget, 1, 0)
+    np.testing.assert_array_equal(pg.counts.cpu().numpy(), po["counts"])
+    k = int(po["counts"].reshape(-1)[0])
+    np.testing.assert_array_equal(pg.idx.cpu().numpy()[..., :k], po["idx"][..., :k])
+    assert np.all(pg.pi_sel.cpu().numpy()[..., :k] == 1.0)
+
+
+def test_plan_overflow_is_reported():
+    B, H, N, d = 1, 1, 1024, 64
+    nkvb = N // 4
+    cfg = abi.Config(kv_block=4, budget=0.05)
+    cap = abi.capacity((B, H, N, d), cfg)
+    pi = torch.ones(B, H, N // 128, nkvb, dtype=torch.float32, device="cuda")
+    pg = abi.plan_from_pi(pi, (B, H, N, d), cfg)
+    with pytest.raises(abi.AbattnError) as e:
+        abi.check()
+    assert e.value.code == abi.ERR_PLAN_OVERFLOW
+    assert np.all(pg.counts.cpu().numpy() == cap)
+    abi.check()  # the error word was cleared
+
+
+# ------------------------------------------------------------------ forward
+
+def _oracle_forward(Q, K, V, plan, kb, rows=None, scale=None):
+    return oracle.forward_rows(Q, K, V, 128, kb, plan.counts.cpu().numpy(), plan.idx.cpu().numpy(),
+                               plan.pi_sel.cpu().numpy(), scale if scale else 1 / math.sqrt(Q.shape[-1]),
+                               rows=rows)
+
+
+def test_sparse_forward_parity_tiny(tiny):
+    cfg = cfg_of(W)
+    plan = abi.plan(tiny["Q"], tiny["K"], cfg)
+    O, lse = abi.forward(tiny["Q"], tiny["K"], tiny["V"], plan, cfg)
+    abi.check()
+    Oo, lo = _oracle_forward(tiny["Qc"], tiny["Kc"], tiny["Vc"], plan, W.kv_block)
+    assert_forward_close(O.float().cpu().numpy(), Oo, "sparse tiny")
+    np.testing.assert_allclose(lse.cpu().numpy(), lo, atol=2e-3, rtol=1e-4)
+
+
+def test_dense_forward_parity_tiny(tiny):
+    O, lse = abi.dense_forward(tiny["Q"], tiny["K"], tiny["V"])
+    abi.check()
+    Qd, Kd, Vd = (oracle.f64(t) for t in (tiny["Qc"], tiny["Kc"], tiny["Vc"]))
+    for h in range(W.H):
+        Oo, lo = oracle.dense(Qd[0, h], Kd[0, h], Vd[0, h], SCALE)
+        assert_forward_close(O[0, h].float().cpu().numpy(), Oo, f"dense h{h}")
+        np.testing.assert_allclose(lse[0, h].cpu().numpy(), lo, atol=2e-3, rtol=1e-4)
+
+
+def test_full_plan_equals_dense(tiny):
+    shape = tuple(tiny["Q"].shape)
+    plan = abi.full_plan(shape, 4)
+    Os, ls = abi.forward(tiny["Q"], tiny["K"], tiny["V"], plan, abi.Config(kv_block=4))
+    Od, ld = abi.dense_forward(tiny["Q"], tiny["K"], tiny["V"])
+    abi.check()
+    assert_forward_close(Os.float().cpu().numpy(), Od.float().cpu().numpy().astype(np.float64), "full vs dense")
+    np.testing.assert_allclose(ls.cpu().numpy(), ld.cpu().numpy(), atol=1e-3)
+
+
+@pytest.mark.parametrize("d,N,kb,budget", [(128, 1000, 4, 0.2), (128, 300, 128, 0.5), (64, 777, 128, 1.0),
+                                           (128, 640, 16, 0.3), (64, 2048, 8, 0.1)])
+def test_sparse_forward_ragged_shapes(d, N, kb, budget):
+    g = torch.Generator().manual_seed(N + kb)
+    Qc, Kc, Vc = (torch.randn(1, 2, N, d, generator=g).to(torch.bfloat16) for _ in range(3))
+    cfg = abi.Config(kv_block=kb, budget=budget, seed=3)
+    Q, K, V = Qc.cuda(), Kc.cuda(), Vc.cuda()
+    plan = abi.plan(Q, K, cfg)
+    O, lse = abi.forward(Q, K, V, plan, cfg)
+    abi.check()
+    Oo, lo = _oracle_forward(Qc, Kc, Vc, plan, kb)
+    assert_forward_close(O.float().cpu().numpy(), Oo, f"d{d} N{N} kb{kb}")
+    np.testing.assert_allclose(lse.cpu().numpy(), lo, atol=2e-3, rtol=1e-4)
+    if N % 128:
+        Od, _ = abi.dense_forward(Q, K, V)
+        abi.check()
+        Oo_d, _ = oracle.dense(Qc[0, 1], Kc[0, 1], Vc[0, 1], 1 / math.sqrt(d))
+        assert_forward_close(Od[0, 1].float().cpu().numpy(), Oo_d, "dense ragged")
+
+
+def test_empty_and_custom_plans():
+    B, H, N, d = 1, 1, 512, 128
+    g = torch.Generator().manual_seed(9)
+    Qc, Kc, Vc = (torch.randn(B, H, N, d, generator=g).to(torch.bfloat16) for _ in range(3))
+    nqb = N // 128
+    cap = 40
+    counts = torch.tensor([[[0, 1, 33, 40]]], dtype=torch.int32)
+    idx = torch.zeros(B, H, nqb, cap, dtype=torch.int32)
+    ps = torch.zeros(B, H, nqb, cap, dtype=torch.float32)
+    rng = np.random.default_rng(1)
+    for qb in range(nqb):
+        n = int(counts[0, 0, qb])
+        sel = np.sort(rng.choice(N // 4, n, replace=False))
+        idx[0, 0, qb, :n] = torch.from_numpy(sel.astype(np.int32))
+        ps[0, 0, qb, :n] = torch.from_numpy(rng.uniform(0.01, 1, n).astype(np.float32))
+    plan = abi.Plan(counts.cuda(), idx.cuda(), ps.cuda(), cap, 4)
+    O, lse = abi.forward(Qc.cuda(), Kc.cuda(), Vc.cuda(), plan, abi.Config(kv_block=4))
+    abi.check()
+    Oo, lo = _oracle_forward(Qc, Kc, Vc, plan, 4)
+    Og = O.float().cpu().numpy()
+    assert np.all(Og[0, 0, :128] == 0) and np.all(np.isneginf(lse[0, 0, :128].cpu().numpy()))
+    assert_forward_close(Og[0, 0, 128:], Oo[0, 0, 128:], "custom plan")
+
+
+def test_bad_plan_index_is_skipped_and_reported():
+    B, H, N, d = 1, 1, 256, 64
+    Q = torch.randn(B, H, N, d, device="cuda").to(torch.bfloat16)
+    counts = torch.tensor([[[2, 1]]], dtype=torch.int32, device="cuda")
+    idx = torch.tensor([[[[3, 10**6], [-5, 0]]]], dtype=torch.int32, device="cuda")
+    ps = torch.ones(1, 1, 2, 2, device="cuda")
+    O, lse = abi.forward(Q, Q, Q, abi.Plan(counts, idx, ps, 2, 4), abi.Config(kv_block=4))
+    with pytest.raises(abi.AbattnError) as e:
+        abi.check()
+    assert e.value.code == abi.ERR_BOUNDS
+    assert torch.isfinite(O[0, 0, :128].float()).all()
+
+
+def test_sip_beats_topk_on_gpu(tiny):
+    """The HT-sampled forward is closer to dense than top-k truncation."""
+    shape = tuple(tiny["Q"].shape)
+    Od, _ = abi.dense_forward(tiny["Q"], tiny["K"], tiny["V"])
+    errs = []
+    for seed in range(8):
+        cfg = cfg_of(W, seed=seed)
+        plan = abi.plan(tiny["Q"], tiny["K"], cfg)
+        O, _ = abi.forward(tiny["Q"], tiny["K"], tiny["V"], plan, cfg)
+        errs.append(((O.float() - Od.float()).norm() / Od.float().norm()).item())
+    cfg = cfg_of(W, mode=abi.MODE_TOPK)
+    plan = abi.plan(tiny["Q"], tiny["K"], cfg)
+    O, _ = abi.forward(tiny["Q"], tiny["K"], tiny["V"], plan, cfg)
+    abi.check()
+    e_top = ((O.float() - Od.float()).norm() / Od.float().norm()).item()
+    print(f"GPU rel-L2 vs dense: SIP {np.mean(errs):.4f}, top-k {e_top:.4f}")
+    assert np.mean(errs) < e_top
