@@ -1,0 +1,436 @@
+#!/usr/bin/env python
+"""AB-Attention hot-path benchmark on B200.
+
+One step = one pass of the whole path over one synthetic layer:
+abattn_plan (mean keys -> k-means -> scores -> water-fill + Poisson
+sampling + compaction) followed by the gathered sparse forward (the plan is
+used by `forwards_per_plan` forwards: 1 for the 14B-like layer, 4 for the
+HunyuanVideo-like one).  The metric is the executed tensor-core TFLOP/s of
+the sparse forward over the step time; the forward alone, every kernel's
+time, the in-house dense kernel and the CPU oracle are reported beside it.
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+        [--workload wan14b-720p|wan1.3b-480p|hunyuan-720p|sweep-75k|tiny]
+For N > 1 launch under torchrun: every rank runs its own full layer (weak
+scaling, no data-path collective; each (b, h, q-block) row is independent).
+"""
+from __future__ import annotations
+
+import argparse
+import concurrent.futures
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from block_sparse_attention_12_b200 import inputs  # noqa: E402
+
+METRIC = "AB-Attn fwd ms & executed TFLOPS (% bf16 TC peak), 75.6K tok × 40 heads"
+UNIT = "TFLOP/s"
+FP32_LANES_PER_SM = 128
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="wan14b-720p", choices=sorted(inputs.WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--dense-iters", type=int, default=3)
+    ap.add_argument("--cpu-rows", type=int, default=64)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm=p["hbm_gbs"], bf16=p["bf16_tflops"], bf16_sus=p["bf16_tflops_sustained"],
+                    sm_mhz=p.get("sm_max_mhz", 1965.0), src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, sm_mhz=1965.0, src="fallback")
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        sel = []
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:
+            pass
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", *sel, f"--query-gpu={self.FIELDS}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.p.terminate()
+        try:
+            self.p.wait(5)
+        except subprocess.TimeoutExpired:
+            self.p.kill()
+        self.f.seek(0)
+        rows = [r.split(",") for r in self.f.read().strip().splitlines() if r.count(",") >= 7]
+        os.unlink(self.f.name)
+        sm, mx, pw, reasons = [], None, [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[0]))
+                mx = float(r[1])
+                pw.append(float(r[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, r[4:8]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        loaded = [s for s, p in zip(sm, pw) if p > 0.3 * max(pw)] if pw else sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- oracle leg
+def oracle_sample(w, n_rows: int, seed_offset: int = 0, n_heads: int = 4):
+    """A bounded seeded sample of rows of the workload: n_rows q-blocks spread
+    over n_heads heads, plus those heads' Q, K, V as float64 (drawn and
+    converted outside any timed region)."""
+    import oracle
+    g = np.random.default_rng(4321 + seed_offset)
+    nqb = math.ceil(w.N / 128)
+    flat_heads = g.choice(w.B * w.H, size=min(n_heads, w.B * w.H), replace=False)
+    heads = [divmod(int(x), w.H) for x in flat_heads]
+    rows = []
+    for i in range(n_rows):
+        b, h = heads[i % len(heads)]
+        rows.append((b, h, int(g.integers(nqb))))
+    data = {bh: tuple(oracle.f64(t) for t in inputs.make_head(w, bh[0], bh[1])) for bh in heads}
+    return rows, data
+
+
+def executed_flops_row(n_sel: int, kb: int, d: int) -> float:
+    return 4.0 * 128 * 128 * d * math.ceil(n_sel * kb / 128)
+
+
+def run_oracle_rows(w, rows, data, threads: int):
+    """Plan + forward of the listed rows with the CPU oracle; returns
+    (seconds, executed-equivalent FLOPs)."""
+    import oracle
+    oracle.set_num_threads(1)
+    t0 = time.perf_counter()
+    kbars = {}
+
+    def kbar(bh):
+        if bh not in kbars:
+            kbars[bh] = oracle.meanpool(data[bh][1], w.kv_block)
+        return kbars[bh]
+
+    for bh in {(b, h) for b, h, _ in rows}:
+        kbar(bh)
+    f64 = data
+
+    def one(r):
+        b, h, qb = r
+        q, k, v = f64[(b, h)]
+        out = oracle.plan_forward_row(q, k, v, kbars[(b, h)], b, h, qb, w.kv_block, w.budget, w.seed,
+                                      w.n_clusters, w.kmeans_iters)
+        flops = executed_flops_row(out["idx"].size, w.kv_block, w.d) * w.forwards_per_plan
+        if w.forwards_per_plan > 1:  # the extra forwards reuse the plan
+            for _ in range(w.forwards_per_plan - 1):
+                oracle.sparse_block(q[qb * 128:qb * 128 + 128], k, v, w.kv_block, out["idx"], out["pi_sel"],
+                                    1 / math.sqrt(w.d))
+        return flops
+
+    with concurrent.futures.ThreadPoolExecutor(threads) as ex:
+        flops = sum(ex.map(one, rows))
+    return time.perf_counter() - t0, flops
+
+
+def cpu_baseline(w, n_rows: int):
+    threads = os.cpu_count() or 1
+    rows, data = oracle_sample(w, n_rows)
+    secs, flops = run_oracle_rows(w, rows, data, threads)
+    return {"value": flops / secs / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{len(rows)} (head, q-block) rows of {w.name} (of {w.B * w.H * math.ceil(w.N / 128)}), "
+                      f"k-means + scores + water-fill + sampling + gathered forward in fp64, "
+                      f"{secs:.2f} s wall on {threads} threads"}
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    threads = os.cpu_count() or 1
+    rows_per_step = max(threads, 16)
+    samples = [oracle_sample(w, rows_per_step, seed_offset=s) for s in range(args.warmup + args.steps)]
+    for s in range(args.warmup):
+        run_oracle_rows(w, *samples[s], threads)
+    tot_s, tot_f = 0.0, 0.0
+    for s in range(args.warmup, args.warmup + args.steps):
+        sec, fl = run_oracle_rows(w, *samples[s], threads)
+        tot_s += sec
+        tot_f += fl
+    value = tot_f / tot_s / 1e12
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "impl": "reference", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": w.name, "tokens": w.N, "heads": w.H, "d": w.d,
+                                           "kv_block": w.kv_block, "budget": w.budget},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": f"each step: {rows_per_step} seeded (head, q-block) rows of {w.name}, "
+                                       f"plan + gathered forward in fp64"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- GPU leg
+def source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "block_sparse_attention_12_b200", "csrc")
+    for n in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel: str, units: float):
+    """DRAM bytes per launch from the committed ncu summary, scaled to this
+    launch's units, if it was captured from the current sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        t = json.load(f)
+    e = t.get(kernel)
+    if not e or e.get("source_hash") != source_hash():
+        return None
+    return e["bytes_per_unit"] * units
+
+
+def timed(fn, iters, stream):
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(iters):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / iters
+
+
+def main():
+    args = parse()
+    w = inputs.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+        return
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    from block_sparse_attention_12_b200 import abi, build
+    build.build()
+    P = peaks()
+    shape = (w.B, w.H, w.N, w.d)
+    Q, K, V = inputs.make_qkv(w, device=f"cuda:{local}", seed=w.seed + 1000 * rank)
+    cfg = abi.Config(kv_block=w.kv_block, budget=w.budget, n_clusters=w.n_clusters,
+                     kmeans_iters=w.kmeans_iters, seed=w.seed)
+    planner = abi.Planner(shape, cfg)
+    O = torch.empty_like(Q)
+    lse = torch.empty(shape[:3], dtype=torch.float32, device=Q.device)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        plan = planner(Q, K)
+        for _ in range(w.forwards_per_plan):
+            abi.forward(Q, K, V, plan, cfg, O=O, lse=lse)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    abi.check()
+    plan = planner.plan
+    exec_fl = abi.executed_flops(plan, shape) * w.forwards_per_plan
+    useful_fl = abi.useful_flops(plan, shape) * w.forwards_per_plan
+
+    # ---- the timed region: K whole steps, barrier + sync on both sides
+    clocks = ClockSampler(local)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    if dist:
+        t = torch.tensor([ms], device=Q.device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    abi.check()
+    value = exec_fl * world / (ms / 1e3) / 1e12
+
+    # ---- per-kernel breakdown (separate loops, same stream, after the timed region)
+    kb_ms = {}
+    n_it = max(3, min(args.steps, 10))
+    Kbar = abi.meanpool(K, w.kv_block)
+    kb_ms["meanpool"] = timed(lambda: abi.meanpool(K, w.kv_block, out=Kbar), n_it, stream)
+    C, wt, _ = abi.kmeans(Q, cfg)
+    kb_ms["kmeans"] = timed(lambda: abi.kmeans(Q, cfg), n_it, stream)
+    S = abi.score(C, wt, Kbar, shape, cfg)
+    kb_ms["score"] = timed(lambda: abi.score(C, wt, Kbar, shape, cfg), n_it, stream)
+    p2 = abi.plan_from_scores(S, shape, cfg)
+    kb_ms["planner"] = timed(lambda: abi.plan_from_scores(S, shape, cfg, plan=p2), n_it, stream)
+    kb_ms["plan_total"] = timed(lambda: planner(Q, K), n_it, stream)
+    kb_ms["forward"] = timed(lambda: abi.forward(Q, K, V, plan, cfg, O=O, lse=lse), n_it, stream)
+    abi.check()
+    del S, p2
+    fwd_fl = abi.executed_flops(plan, shape)
+    fwd_tf = fwd_fl / (kb_ms["forward"] / 1e3) / 1e12
+
+    dense = None
+    if not args.no_dense and rank == 0:
+        Od = torch.empty_like(Q)
+        abi.dense_forward(Q, K, V, O=Od, want_lse=False)
+        dms = timed(lambda: abi.dense_forward(Q, K, V, O=Od, want_lse=False), args.dense_iters, stream)
+        abi.check()
+        dfl = 4.0 * w.B * w.H * w.N * w.N * w.d
+        dense = {"ms": dms, "tflops": dfl / (dms / 1e3) / 1e12, "frac_of_bf16_peak": dfl / (dms / 1e3) / 1e12 / P["bf16"]}
+        del Od
+
+    # ---- rooflines (algorithmic work per launch / measured launch time)
+    BH = w.B * w.H
+    nqb, nkvb = math.ceil(w.N / 128), math.ceil(w.N / w.kv_block)
+    rows = BH * nqb
+    sel_cnt = float(plan.counts.sum().item())
+    fp32_peak = 148 * FP32_LANES_PER_SM * 2 * P["sm_mhz"] * 1e6 / 1e12
+    roofs = {
+        "forward": {"bound": "tensor", "achieved": fwd_tf, "peak": P["bf16"], "unit": "TFLOP/s",
+                    "work": fwd_fl, "traffic": traffic_for("forward", rows)},
+        "meanpool": {"bound": "hbm", "unit": "GB/s", "peak": P["hbm"],
+                     "work": BH * w.N * w.d * 2 + BH * nkvb * w.d * 4,
+                     "traffic": traffic_for("meanpool", BH * nkvb)},
+        "kmeans": {"bound": "alu", "unit": "TFLOP/s", "peak": fp32_peak,
+                   "work": rows * w.kmeans_iters * (128 * 8 * w.d * 3 + 128 * w.d * 8 * 2),
+                   "traffic": traffic_for("kmeans", rows)},
+        "score": {"bound": "alu", "unit": "TFLOP/s", "peak": fp32_peak,
+                  "work": 2 * (2.0 * rows * 8 * nkvb * w.d), "traffic": traffic_for("score", rows)},
+        "planner": {"bound": "hbm", "unit": "GB/s", "peak": P["hbm"],
+                    "work": rows * nkvb * 4 + rows * 4 + sel_cnt * 8, "traffic": traffic_for("planner", rows)},
+    }
+    for k, r in roofs.items():
+        t = kb_ms[k] / 1e3
+        if k != "forward":
+            r["achieved"] = r["work"] / t / (1e9 if r["unit"] == "GB/s" else 1e12)
+        r["frac"] = r["achieved"] / r["peak"]
+        r["ms"] = kb_ms[k]
+    step_share = {k: kb_ms[k] * (w.forwards_per_plan if k == "forward" else 1) for k in roofs}
+    dom = max(step_share, key=step_share.get)
+    rd = roofs[dom]
+    roofline = {"kernel": dom, "bound": rd["bound"], "achieved": rd["achieved"], "peak": rd["peak"],
+                "unit": rd["unit"], "frac": rd["frac"], "traffic": rd["traffic"],
+                "peak_source": P["src"] + (" bf16 burst" if rd["bound"] == "tensor" else
+                                           (" hbm copy" if rd["bound"] == "hbm" else
+                                            " fp32 lanes x 2 x max SM clock (derived)"))}
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        Qh, Kh, Vh = (t.cpu().pin_memory() for t in (Q, K, V))
+        Oh = torch.empty(O.shape, dtype=O.dtype, pin_memory=True)
+        Qd, Kd, Vd = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
+
+        def e2e_step():
+            Qd.copy_(Qh, non_blocking=True)
+            Kd.copy_(Kh, non_blocking=True)
+            Vd.copy_(Vh, non_blocking=True)
+            pl = planner(Qd, Kd)
+            for _ in range(w.forwards_per_plan):
+                abi.forward(Qd, Kd, Vd, pl, cfg, O=O, lse=lse)
+            Oh.copy_(O, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+        e2e_ms = timed(e2e_step, args.e2e_steps, stream)
+        if dist:
+            t = torch.tensor([e2e_ms], device=Q.device)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        abi.check()
+        e2e = {"value": exec_fl * world / (e2e_ms / 1e3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": 3 * Q.numel() * Q.element_size(),
+               "d2h_bytes_per_step": O.numel() * O.element_size()}
+        del Qh, Kh, Vh, Oh, Qd, Kd, Vd
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, args.cpu_rows)
+
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "tokens": w.N, "heads": w.H, "d": w.d, "grid": list(w.grid),
+                   "kv_block": w.kv_block, "budget": w.budget, "q_block": 128, "clusters": w.n_clusters,
+                   "kmeans_iters": w.kmeans_iters, "forwards_per_plan": w.forwards_per_plan,
+                   "step": "abattn_plan + forwards_per_plan x abattn_forward",
+                   "l2": "inputs larger than L2 (Q, K, V %.2f GB per GPU)" % (3 * Q.numel() * 2 / 1e9),
+                   "parallelism": f"weak x{world}: one full layer per GPU"},
+        "fwd_ms": kb_ms["forward"], "fwd_tflops": fwd_tf, "fwd_frac_of_bf16_peak": fwd_tf / P["bf16"],
+        "plan_ms": kb_ms["plan_total"], "kernel_ms": kb_ms,
+        "executed_tflop_per_step": exec_fl / 1e12, "useful_tflop_per_step": useful_fl / 1e12,
+        "selected_blocks_mean": sel_cnt / rows, "sparsity": 1.0 - sel_cnt / rows / nkvb,
+        "dense": dense, "roofline": roofline,
+        "rooflines": {k: {kk: vv for kk, vv in r.items() if kk != "work"} for k, r in roofs.items()},
+        "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
+        "gpu_launches": 7 * args.steps if w.forwards_per_plan == 1 else (6 + w.forwards_per_plan) * args.steps,
+        "peaks": P,
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

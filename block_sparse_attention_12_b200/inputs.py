@@ -8,8 +8,8 @@ Recipe (AB-Attention news write-up, section "how it was measured": Wan2.1 at
 81 frames and HunyuanVideo at 129 frames, 720p latents; the sweep shape is the
 75,600-token x 10-head x d128 workload of the Splash-attention page, Table 2):
 
-* Q, K, V are drawn, in that order, as float32 N(0, 1) of shape [B, H, N, d]
-  from one seeded generator.
+* Q, K, V are drawn as float32 N(0, 1), one PCG64 stream per (seed, batch,
+  head, tensor), so that any single head can be rebuilt on its own.
 * Token n is the frame-major (F, H, W) position n = (f * Hg + y) * Wg + x.
   A shared 3D sinusoidal code p[n] is added, scaled by 0.8, to Q, K and V of
   every batch and head.  p concatenates, for each axis a in (f, y, x),
@@ -21,9 +21,12 @@ Recipe (AB-Attention news write-up, section "how it was measured": Wan2.1 at
 """
 from __future__ import annotations
 
+import concurrent.futures
 import dataclasses
 import math
+import os
 
+import numpy as np
 import torch
 
 
@@ -85,30 +88,56 @@ def position_code(grid, d: int) -> torch.Tensor:
     return out.to(torch.float32)
 
 
-def make_qkv(w: Workload, device: str = "cpu", seed: int | None = None):
-    """Return bf16 Q, K, V of shape [B, H, N, d] on `device`.
+def _stream(seed: int, *key: int) -> np.random.Generator:
+    return np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, *key])))
 
-    The draw happens on `device` with a generator seeded by `seed`
-    (default: the workload's).  A CPU draw is reproducible everywhere; a CUDA
-    draw is reproducible on the same GPU model and is used for the large
-    layers, whose CPU draw would take minutes.
-    """
+
+def outlier_rows(w: Workload, seed: int | None = None) -> np.ndarray:
+    """Token rows whose Q, K, V are scaled by the outlier factor."""
     seed = w.seed if seed is None else seed
-    g = torch.Generator(device=device)
-    g.manual_seed(seed)
-    shape = (w.B, w.H, w.N, w.d)
-    pos = (0.8 * position_code(w.grid, w.d)).to(device)
+    if w.outlier_frac <= 0:
+        return np.zeros(0, dtype=np.int64)
+    n_out = int(round(w.outlier_frac * w.N))
+    return np.sort(_stream(seed, 0x0071E5).permutation(w.N)[:n_out])
+
+
+def make_head(w: Workload, b: int, h: int, seed: int | None = None, pos=None, rows=None):
+    """Q, K, V of one (batch, head) as bf16 [N, d] CPU tensors.
+
+    Each of the three tensors of each head has its own PCG64 stream keyed
+    by (seed, b, h, tensor), so any head can be rebuilt alone."""
+    seed = w.seed if seed is None else seed
+    pos = (0.8 * position_code(w.grid, w.d)).numpy() if pos is None else pos
+    rows = outlier_rows(w, seed) if rows is None else rows
     out = []
-    for _ in range(3):
-        t = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
-        t += pos
-        out.append(t)
-    if w.outlier_frac > 0:
-        n_out = int(round(w.outlier_frac * w.N))
-        rows = torch.randperm(w.N, generator=g, device=device)[:n_out]
-        for t in out:
-            t[:, :, rows, :] *= w.outlier_scale
-    return tuple(t.to(torch.bfloat16).contiguous() for t in out)
+    for t in range(3):
+        x = _stream(seed, b, h, t).standard_normal((w.N, w.d), dtype=np.float32)
+        x += pos
+        if rows.size:
+            x[rows] *= np.float32(w.outlier_scale)
+        out.append(torch.from_numpy(x).to(torch.bfloat16))
+    return tuple(out)
+
+
+def make_qkv(w: Workload, device: str = "cpu", seed: int | None = None, threads: int | None = None):
+    """Return bf16 Q, K, V of shape [B, H, N, d] on `device` (drawn on the
+    host, one head per task in a thread pool; identical on every machine)."""
+    seed = w.seed if seed is None else seed
+    pos = (0.8 * position_code(w.grid, w.d)).numpy()
+    rows = outlier_rows(w, seed)
+    Q, K, V = (torch.empty(w.B, w.H, w.N, w.d, dtype=torch.bfloat16) for _ in range(3))
+
+    def one(bh):
+        b, h = divmod(bh, w.H)
+        q, k, v = make_head(w, b, h, seed, pos, rows)
+        Q[b, h], K[b, h], V[b, h] = q, k, v
+
+    threads = threads or min(32, os.cpu_count() or 1)
+    with concurrent.futures.ThreadPoolExecutor(threads) as ex:
+        list(ex.map(one, range(w.B * w.H)))
+    if device != "cpu":
+        Q, K, V = (t.to(device) for t in (Q, K, V))
+    return Q, K, V
 
 
 def row_sample(w: Workload, n_rows: int, seed: int = 1234):

@@ -77,7 +77,11 @@ def f64(x) -> np.ndarray:
     try:
         import torch
         if isinstance(x, torch.Tensor):
-            return np.ascontiguousarray(x.detach().to("cpu", torch.float64).numpy())
+            x = x.detach().to("cpu")
+            if x.dtype == torch.bfloat16:  # exact: a bf16 is the top half of an fp32
+                bits = x.contiguous().view(torch.int16).numpy().astype(np.uint32) << 16
+                return np.ascontiguousarray(bits.view(np.float32).astype(np.float64))
+            return np.ascontiguousarray(x.to(torch.float64).numpy())
     except ImportError:  # pragma: no cover
         pass
     return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
@@ -251,3 +255,28 @@ def forward_rows(Q, K, V, qblk: int, kb: int, counts, idx, pi_sel, scale: float,
     lib().oc_forward_rows(Q, K, V, B * H, N, d, qblk, kb, rp, n_rows, counts, idx, pi_sel, cap,
                           scale, O, lse)
     return O, lse
+
+
+def plan_forward_row(Qh, Kh, Vh, Kbar_h, b: int, h: int, qb: int, kb: int, budget: float, seed: int,
+                     nc: int = 8, iters: int = 10, scale: float | None = None, mode: int = 0):
+    """The whole path for one q-block row of one head, step by step:
+    k-means of the row's queries, scores against the head's mean keys,
+    water-fill + Poisson sampling (or top-k), then the gathered forward.
+    Qh, Kh, Vh: float64 [N, d] of the head; Kbar_h: its mean keys.
+    Returns dict(O, lse, idx, pi_sel, S)."""
+    Qh, Kh, Vh = f64(Qh), f64(Kh), f64(Vh)
+    N, d = Qh.shape
+    scale = 1.0 / (d ** 0.5) if scale is None else scale
+    q0 = qb * 128
+    Qb = np.ascontiguousarray(Qh[q0:q0 + 128])
+    C, w, _ = kmeans(Qb, nc, iters)
+    s = scores(C, w, Kbar_h, scale)
+    nkvb = s.size
+    if mode == 0:
+        pi, _, _ = waterfill(s, budget * nkvb)
+        idx, ps, _ = sample(pi.astype(np.float32), seed, b, h, qb)
+    else:
+        idx = topk(s, int(np.floor(budget * nkvb + 0.5)))
+        ps = np.ones(idx.size, dtype=np.float32)
+    O, lse = sparse_block(Qb, Kh, Vh, kb, idx, ps, scale)
+    return dict(O=O, lse=lse, idx=idx, pi_sel=ps, S=s)
