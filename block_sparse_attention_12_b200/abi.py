@@ -26,8 +26,9 @@ EXPORTED = [
     "abattn_version", "abattn_strerror", "abattn_check", "abattn_plan_capacity",
     "abattn_plan_workspace_size", "abattn_score_workspace_size", "abattn_meanpool",
     "abattn_kmeans", "abattn_score", "abattn_plan_from_scores", "abattn_plan_from_pi",
-    "abattn_plan", "abattn_forward", "abattn_dense_forward",
+    "abattn_plan", "abattn_forward", "abattn_dense_forward", "abattn_plan_noalloc",
 ]
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class Dims(ctypes.Structure):
@@ -76,6 +77,7 @@ def lib():
         L.abattn_plan.argtypes = [VP, VP, P_D, P_P, VP, VP, VP, ctypes.c_int64, VP, ctypes.c_size_t, VP]
         L.abattn_forward.argtypes = [VP, VP, VP, P_D, P_P, VP, VP, VP, ctypes.c_int64, VP, VP, VP]
         L.abattn_dense_forward.argtypes = [VP, VP, VP, P_D, ctypes.c_float, VP, VP, VP]
+        L.abattn_plan_noalloc.argtypes = [VP, VP, P_D, P_P, VP, VP, VP, ctypes.c_int64, VP]
         for name in EXPORTED:
             if name not in ("abattn_version", "abattn_strerror"):
                 getattr(L, name).restype = ctypes.c_int
@@ -247,6 +249,19 @@ class Planner:
 
 def plan(Q, K, cfg: Config, stream=None) -> Plan:
     return Planner(Q.shape, cfg, Q.device)(Q, K, stream)
+
+
+def plan_noalloc(Q, K, cfg: Config, plan: Plan | None = None, stream=None) -> Plan:
+    """abattn_plan_noalloc: the same plan as `plan`, with the library's own
+    fixed scratch array instead of a caller workspace (small layers only).
+    The output buffers are still the caller's (allocated here when `plan` is
+    None)."""
+    _check_qkv(Q, K)
+    p = empty_plan(Q.shape, cfg, Q.device) if plan is None else plan
+    _ok(lib().abattn_plan_noalloc(_ptr(Q), _ptr(K), ctypes.byref(dims_of(Q)), ctypes.byref(cfg.params()),
+                                  _ptr(p.counts), _ptr(p.idx), _ptr(p.pi_sel), p.cap, _stream(stream)),
+        "abattn_plan_noalloc")
+    return p
 
 
 def forward(Q, K, V, plan: Plan, cfg: Config | None = None, O=None, lse=None, want_lse=True, stream=None):

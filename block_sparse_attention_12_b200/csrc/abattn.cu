@@ -466,3 +466,54 @@ int abattn_dense_forward(const void *Q, const void *K, const void *V, const abat
 }
 
 }  // extern "C"
+
+// ====================================================================== allocation-free plan
+// A variant of abattn_plan whose scratch (mean keys, centroids, weights,
+// scores and score statistics) lives in a fixed array compiled into this
+// library, for callers that may not allocate device memory themselves.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB per device, held until exit
+
+static __device__ __align__(256) unsigned char g_plan_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void *g_scratch_addr[kMaxDevices] = {};
+
+// Device address of g_plan_scratch on the current device.  The name of the
+// array is only a host-side stand-in; the address comes from
+// cudaGetSymbolAddress, looked up once per device with that device current.
+int scratch_address(void **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_status(e);
+    if (dev < 0 || dev >= kMaxDevices) return ABATTN_ERR_DEVICE;
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (g_scratch_addr[dev] == nullptr) {
+        void *ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, g_plan_scratch);
+        if (e != cudaSuccess) return cuda_status(e);
+        g_scratch_addr[dev] = ptr;
+    }
+    *out = g_scratch_addr[dev];
+    return ABATTN_OK;
+}
+
+}  // namespace
+
+extern "C" int abattn_plan_noalloc(const void *Q, const void *K, const abattn_dims *dims, const abattn_params *p,
+                                   int32_t *counts, int32_t *idx, float *pi_sel, int64_t cap, void *stream) {
+    int rc = check_dims(dims);
+    if (rc) return rc;
+    if ((rc = check_params(p, true))) return rc;
+    if (carve(nullptr, dims, p).bytes > kNoAllocScratchBytes) return ABATTN_ERR_WORKSPACE;
+    if (Q == nullptr || K == nullptr || counts == nullptr || idx == nullptr || pi_sel == nullptr)
+        return ABATTN_ERR_NULL;
+    if ((rc = check_device())) return rc;
+    void *scratch = nullptr;
+    if ((rc = scratch_address(&scratch))) return rc;
+    // Every byte of the scratch that the plan reads is written earlier in the
+    // same call, so nothing has to be cleared between calls.
+    return abattn_plan(Q, K, dims, p, counts, idx, pi_sel, cap, scratch, kNoAllocScratchBytes, stream);
+}

@@ -162,6 +162,30 @@ int abattn_forward(const void *Q, const void *K, const void *V, const abattn_dim
 int abattn_dense_forward(const void *Q, const void *K, const void *V, const abattn_dims *dims,
                          float scale, void *O, float *lse, void *stream);
 
+/* Allocation-free variant of abattn_plan.  The paper has no counterpart:
+ * this is a convenience of this library.  Some callers cannot allocate
+ * device memory, for instance a host whose runtime owns all device memory
+ * through its own pool and forbids other allocations, or code that must not
+ * allocate while it runs.  This entry point needs no workspace argument:
+ * its scratch is an array of ABATTN_NOALLOC_SCRATCH_BYTES compiled into the
+ * library, which every GPU that loads the library holds until the process
+ * exits.  Inputs and outputs are the caller's, as for abattn_plan, and the
+ * results are the same.
+ *  - Problems whose plan scratch (abattn_plan_workspace_size) exceeds
+ *    ABATTN_NOALLOC_SCRATCH_BYTES are rejected with ABATTN_ERR_WORKSPACE
+ *    before anything is launched.
+ *  - The first call on a device looks up the scratch array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - All calls on a device share the one array and it keeps the last call's
+ *    contents (nothing in it needs clearing: every value read is written
+ *    earlier in the same call).  Calls that overlap on the GPU, e.g. on two
+ *    streams at once, race on the array and must be serialised by the caller.
+ *  - Never calls cudaMalloc, cudaFree or any allocating routine. */
+#define ABATTN_NOALLOC_SCRATCH_BYTES (32u << 20)
+int abattn_plan_noalloc(const void *Q, const void *K, const abattn_dims *dims, const abattn_params *p,
+                        int32_t *counts, int32_t *idx, float *pi_sel, int64_t cap, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
