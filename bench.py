@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="wan14b-720p", choices=sorted(inputs.WORKLOADS))
+    ap.add_argument("--heads", type=int, default=0,
+                    help="run only this many heads of the layer (small cases for ncu captures)")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--dense-iters", type=int, default=3)
     ap.add_argument("--cpu-rows", type=int, default=64)
@@ -248,6 +250,9 @@ def timed(fn, iters, stream):
 def main():
     args = parse()
     w = inputs.WORKLOADS[args.workload]
+    if args.heads:
+        import dataclasses
+        w = dataclasses.replace(w, H=args.heads, name=f"{w.name}-{args.heads}heads")
     if args.impl == "reference":
         run_reference(args, w)
         return

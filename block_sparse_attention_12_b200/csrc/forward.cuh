@@ -11,19 +11,25 @@
 // One CTA per 128-query block, 192 threads, warp-specialised:
 //   warp 0      producer: TMA of the Q tile once; per 128-key tile, the
 //               selected KV blocks' K and V rows (one kb-row box per block and
-//               64-column half, 128-byte swizzle) and the tile's per-key
-//               log2(1/pi) bias into shared memory;
-//   warp 1      TMEM owner and MMA issuer: S = Q K^T into one of two TMEM
-//               buffers (128 columns each), O += P V into a third (d columns),
+//               64-column half, 128-byte swizzle, 3 stages) and the tile's
+//               per-key log2(1/pi) bias into shared memory.  Each lane owns
+//               one block slot of the tile and fetches the plan entries of
+//               the next tile while the current one is in flight;
+//   warp 1      TMEM owner and MMA issuer: S = Q K^T (both operands in shared
+//               memory) into one of two TMEM buffers of 128 columns; O += P V
+//               with P read from TMEM (it overwrites the first 64 columns of
+//               its S buffer as packed bf16) and V from shared memory;
 //               tcgen05.commit to mbarriers;
 //   warps 2..5  softmax: one query row per thread (TMEM lane); logits
 //               t = s * scale * log2(e) + log2(1/pi); running max with lazy
 //               O rescaling (only when the max grows by more than 2^8);
-//               P = exp2(t - m) as bf16 into a swizzled shared-memory tile;
-//               the epilogue normalises O and writes O (bf16) and the
+//               P = exp2(t - m) packed to bf16 and stored back to TMEM; the
+//               epilogue normalises O and writes O (bf16) and the
 //               natural-log LSE.
 // The MMA warp issues QK^T of tile t+1 before PV of tile t, so the softmax
-// of one tile overlaps the tensor-core work of its neighbours.
+// of one tile overlaps the tensor-core work of its neighbours; MMAs issued
+// by one thread run in order, so QK^T of tile t+2 cannot overwrite P(t)
+// before PV(t) has read it.
 #pragma once
 
 #include "common.cuh"
@@ -31,7 +37,7 @@
 namespace abattn {
 
 constexpr int FWD_THREADS = 192;
-constexpr int FWD_NS = 2;  // K/V stages
+constexpr int FWD_NS = 3;  // K/V stages
 constexpr uint32_t FWD_TMEM_COLS = 512;
 constexpr uint32_t FWD_TMEM_O = 256;  // O accumulator column offset
 
@@ -56,10 +62,9 @@ struct FwdLayout {
     static constexpr int Q_OFF = 0;
     static constexpr int K_OFF = Q_OFF + TILE;
     static constexpr int V_OFF = K_OFF + FWD_NS * TILE;
-    static constexpr int P_OFF = V_OFF + FWD_NS * TILE;
-    static constexpr int BIAS_OFF = P_OFF + 32768;
+    static constexpr int BIAS_OFF = V_OFF + FWD_NS * TILE;
     static constexpr int BAR_OFF = BIAS_OFF + FWD_NS * 128 * 4;
-    static constexpr int NBARS = 1 + 2 * FWD_NS + 6;
+    static constexpr int NBARS = 1 + 2 * FWD_NS + 4;
     static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
     static constexpr int BYTES = MISC_OFF + 16;
     static constexpr int ALLOC = BYTES + 1024;  // slack for 1024-byte alignment
@@ -85,15 +90,13 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
     uint8_t *sQ = smem + L::Q_OFF;
     uint8_t *sK = smem + L::K_OFF;
     uint8_t *sV = smem + L::V_OFF;
-    uint8_t *sP = smem + L::P_OFF;
     float *sBias = reinterpret_cast<float *>(smem + L::BIAS_OFF);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::BAR_OFF);
     uint64_t *q_full = bars;
     uint64_t *kv_full = bars + 1;
     uint64_t *kv_empty = bars + 1 + FWD_NS;
     uint64_t *s_full = bars + 1 + 2 * FWD_NS;
-    uint64_t *s_free = s_full + 2;
-    uint64_t *p_full = s_free + 2;
+    uint64_t *p_full = s_full + 2;
     uint64_t *pv_done = p_full + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::MISC_OFF);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::MISC_OFF + 4);
@@ -119,10 +122,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
             mbar_init(&kv_full[s], 1);
             mbar_init(&kv_empty[s], 1);
         }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&s_full[i], 1);
-            mbar_init(&s_free[i], 4);
-        }
+        for (int i = 0; i < 2; ++i) mbar_init(&s_full[i], 1);
         mbar_init(p_full, 4);
         mbar_init(pv_done, 1);
         *abort_flag = 0;
@@ -153,35 +153,50 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
             }
             const int32_t *ridx = DENSE ? nullptr : p.idx + int64_t(row) * p.cap;
             const float *rpi = DENSE ? nullptr : p.pi_sel + int64_t(row) * p.cap;
-            const int spt = DENSE ? 1 : 128 / p.kb;  // KV blocks per 128-key tile
+            const int spt = DENSE ? 1 : 128 / p.kb;  // KV blocks per 128-key tile (<= 32)
             int fill_blk = 0;                       // a valid block to load into padding slots
             if (!DENSE) {
                 const int b0 = ridx[0];
                 fill_blk = (b0 >= 0 && b0 < p.nkvb) ? b0 : 0;
             }
+            // plan entries of this lane's slot in tile t (prefetched one tile ahead)
+            auto fetch = [&](int t, int &blk, float &pi) {
+                const int slot = t * spt + lane;
+                blk = -1;
+                pi = 0.f;
+                if (!DENSE && lane < spt && slot < cnt) {
+                    blk = __ldg(ridx + slot);
+                    pi = __ldg(rpi + slot);
+                }
+            };
+            int cur_blk, nxt_blk;
+            float cur_pi, nxt_pi;
+            fetch(0, cur_blk, cur_pi);
             for (int t = 0; t < T; ++t) {
                 const int s = t % FWD_NS;
+                fetch(t + 1, nxt_blk, nxt_pi);
                 if (t >= FWD_NS && !mbar_wait(&kv_empty[s], ((t / FWD_NS) - 1) & 1, abort_flag)) break;
-                // per-key bias of this tile: log2(1/pi) of the key's block, -inf if absent
+                // this lane's slot: valid block and its bias
+                bool mine_ok = false;
+                float mine_b = -INFINITY;
+                if (!DENSE && lane < spt && t * spt + lane < cnt) {
+                    mine_ok = cur_blk >= 0 && cur_blk < p.nkvb && cur_pi > 0.f;
+                    if (mine_ok) mine_b = -log2f(cur_pi);
+                    else raise_error(kErrBounds);
+                }
+                // bias of keys 4*lane .. 4*lane+3 (all in one block since kb >= 4)
                 float bv[4];
+                if (DENSE) {
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int pos = lane * 4 + i;
-                    if (DENSE) {
-                        bv[i] = (t * 128 + pos < p.N) ? 0.f : -INFINITY;
-                    } else {
-                        const int slot = t * spt + pos / p.kb;
-                        bv[i] = -INFINITY;
-                        if (slot < cnt) {
-                            const int blk = ridx[slot];
-                            const float pi = rpi[slot];
-                            if (blk < 0 || blk >= p.nkvb || !(pi > 0.f)) {
-                                raise_error(kErrBounds);
-                            } else {
-                                const int key = blk * p.kb + pos % p.kb;
-                                if (key < p.N) bv[i] = -log2f(pi);
-                            }
-                        }
+                    for (int i = 0; i < 4; ++i) bv[i] = (t * 128 + lane * 4 + i < p.N) ? 0.f : -INFINITY;
+                } else {
+                    const int owner = (lane * 4) / p.kb;
+                    const float b = __shfl_sync(0xffffffffu, mine_b, owner);
+                    const int blk = __shfl_sync(0xffffffffu, cur_blk, owner);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int key = blk * p.kb + (lane * 4 + i) % p.kb;
+                        bv[i] = key < p.N ? b : -INFINITY;
                     }
                 }
                 *reinterpret_cast<float4 *>(sBias + s * 128 + lane * 4) = make_float4(bv[0], bv[1], bv[2], bv[3]);
@@ -198,20 +213,17 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                             tma_load_3d(dV + h * 16384, &tmV, &kv_full[s], h * 64, t * 128, bh);
                         }
                     }
-                } else {
-                    for (int q = lane; q < spt; q += 32) {
-                        const int slot = t * spt + q;
-                        int blk = slot < cnt ? ridx[slot] : fill_blk;
-                        if (blk < 0 || blk >= p.nkvb) blk = fill_blk;
-                        const int r0 = blk * p.kb;
-                        const int off = q * p.kb * 128;  // kb rows of 128 bytes per half
+                } else if (lane < spt) {
+                    const int r0 = (mine_ok ? cur_blk : fill_blk) * p.kb;
+                    const int off = lane * p.kb * 128;  // kb rows of 128 bytes per half
 #pragma unroll
-                        for (int h = 0; h < L::HALVES; ++h) {
-                            tma_load_3d(dK + h * 16384 + off, &tmK, &kv_full[s], h * 64, r0, bh);
-                            tma_load_3d(dV + h * 16384 + off, &tmV, &kv_full[s], h * 64, r0, bh);
-                        }
+                    for (int h = 0; h < L::HALVES; ++h) {
+                        tma_load_3d(dK + h * 16384 + off, &tmK, &kv_full[s], h * 64, r0, bh);
+                        tma_load_3d(dV + h * 16384 + off, &tmV, &kv_full[s], h * 64, r0, bh);
                     }
                 }
+                cur_blk = nxt_blk;
+                cur_pi = nxt_pi;
                 ++issued;
             }
             // drain: every issued copy lands before the CTA may exit
@@ -228,12 +240,11 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         if (lane == 0 && T > 0) {
             constexpr uint32_t idesc_qk = make_idesc_bf16(128, 128, 0, 0);
             constexpr uint32_t idesc_pv = make_idesc_bf16(128, HD, 0, 1);
-            const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
+            const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
             bool ok = mbar_wait(q_full, 0, abort_flag);
             auto issue_qk = [&](int t) -> bool {
                 const int s = t % FWD_NS, sb = t & 1;
                 if (!mbar_wait(&kv_full[s], (t / FWD_NS) & 1, abort_flag)) return false;
-                if (t >= 2 && !mbar_wait(&s_free[sb], ((t >> 1) - 1) & 1, abort_flag)) return false;
                 tc_fence_after();
                 const uint32_t kbase = aK + s * L::TILE;
 #pragma unroll
@@ -252,10 +263,10 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                 tc_fence_after();
                 const int s = t % FWD_NS;
                 const uint32_t vbase = aV + s * L::TILE;
+                const uint32_t pbase = tmem + (t & 1) * 128;
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
-                    umma_f16_ss(tmem + FWD_TMEM_O,
-                                make_sdesc_sw128(aP + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024),
+                    umma_f16_ts(tmem + FWD_TMEM_O, pbase + k * 8,
                                 make_sdesc_sw128(vbase + k * 2048, 16384, 1024), idesc_pv,
                                 (t > 0 || k > 0) ? 1u : 0u);
                 }
@@ -283,9 +294,6 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
 #pragma unroll
             for (int c = 0; c < 4; ++c) tmem_ld32(t_lane + sb * 128 + c * 32, x[c]);
             tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s_free[sb]);
 
             const float *bias = sBias + s * 128;
             float mt = -INFINITY;
@@ -342,20 +350,18 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                     tmem_wait_st();
                 }
             }
-            // P row -> shared memory, K-major 128-byte-swizzled (two 64-key halves)
-            uint8_t *prow = sP + (rr >> 3) * 1024 + (rr & 7) * 128;
+            // P row -> TMEM, packed bf16 pairs over the first 64 columns of this S buffer
 #pragma unroll
-            for (int c8 = 0; c8 < 16; ++c8) {
-                const int c = c8 >> 2, i0 = (c8 & 3) * 8;
-                uint4 v;
-                v.x = pack_bf16x2(__uint_as_float(x[c][i0 + 0]), __uint_as_float(x[c][i0 + 1]));
-                v.y = pack_bf16x2(__uint_as_float(x[c][i0 + 2]), __uint_as_float(x[c][i0 + 3]));
-                v.z = pack_bf16x2(__uint_as_float(x[c][i0 + 4]), __uint_as_float(x[c][i0 + 5]));
-                v.w = pack_bf16x2(__uint_as_float(x[c][i0 + 6]), __uint_as_float(x[c][i0 + 7]));
-                const int h = c8 >> 3, cc = c8 & 7;
-                *reinterpret_cast<uint4 *>(prow + h * 16384 + ((cc ^ (rr & 7)) << 4)) = v;
+            for (int c = 0; c < 4; c += 2) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    pk[i] = pack_bf16x2(__uint_as_float(x[c][2 * i]), __uint_as_float(x[c][2 * i + 1]));
+                    pk[16 + i] = pack_bf16x2(__uint_as_float(x[c + 1][2 * i]), __uint_as_float(x[c + 1][2 * i + 1]));
+                }
+                tmem_st32(t_lane + sb * 128 + c * 16, pk);
             }
-            fence_proxy_async_smem();
+            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(p_full);
