@@ -354,8 +354,9 @@ def main():
         "kmeans": {"bound": "alu", "unit": "TFLOP/s", "peak": fp32_peak,
                    "work": rows * w.kmeans_iters * (128 * 8 * w.d * 3 + 128 * w.d * 8 * 2),
                    "traffic": traffic_for("kmeans", rows)},
-        "score": {"bound": "alu", "unit": "TFLOP/s", "peak": fp32_peak,
-                  "work": 2 * (2.0 * rows * 8 * nkvb * w.d), "traffic": traffic_for("score", rows)},
+        # tensor cores, bf16 hi/lo split: 3 MMAs per product, 2 passes over 8 cluster slots
+        "score": {"bound": "tensor", "unit": "TFLOP/s", "peak": P["bf16"],
+                  "work": 3 * 2 * (2.0 * rows * 8 * nkvb * w.d), "traffic": traffic_for("score", rows)},
         "planner": {"bound": "hbm", "unit": "GB/s", "peak": P["hbm"],
                     "work": rows * nkvb * 4 + rows * 4 + sel_cnt * 8, "traffic": traffic_for("planner", rows)},
     }

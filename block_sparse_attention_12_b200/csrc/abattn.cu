@@ -72,19 +72,25 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// 3D view {d, N, B*H} of a bf16 [B][H][N][d] tensor; box {64, rows, 1},
-// 128-byte swizzle, zero fill outside the tensor (rows past N).
-int make_map(CUtensorMap *m, const void *base, const abattn_dims *d, int box_rows) {
+// 3D view {d, rows, batches} of a bf16 [batches][rows][d] tensor; box
+// {64, box_rows, 1}, 128-byte swizzle, zero fill outside the tensor (so a
+// tile past the last row never reads the next batch).
+int make_map_rows(CUtensorMap *m, const void *base, int64_t d, int64_t rows, int64_t batches, int box_rows) {
     auto fn = encode_fn();
     if (fn == nullptr) return ABATTN_ERR_DEVICE;
-    cuuint64_t dims[3] = {cuuint64_t(d->d), cuuint64_t(d->N), cuuint64_t(d->B * d->H)};
-    cuuint64_t strides[2] = {cuuint64_t(d->d * 2), cuuint64_t(d->N * d->d * 2)};
+    cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(rows), cuuint64_t(batches)};
+    cuuint64_t strides[2] = {cuuint64_t(d * 2), cuuint64_t(rows * d * 2)};
     cuuint32_t box[3] = {64u, cuuint32_t(box_rows), 1u};
     cuuint32_t estr[3] = {1u, 1u, 1u};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
                     estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? ABATTN_OK : ABATTN_ERR_CUDA;
+}
+
+// Q, K, V [B][H][N][d] as {d, N, B*H}.
+int make_map(CUtensorMap *m, const void *base, const abattn_dims *d, int box_rows) {
+    return make_map_rows(m, base, d->d, d->N, d->B * d->H, box_rows);
 }
 
 int check_device() {
@@ -103,23 +109,17 @@ int sm_count() {
     return n;
 }
 
+// Plan workspace: mean keys and centroids as bf16 hi/lo pairs (the score
+// kernel's operands), cluster weights, scores.
 struct PlanWs {
-    float *Kbar, *C, *w, *S;
-    float2 *partials, *stats;
+    __nv_bfloat16 *Khi, *Klo, *Chi, *Clo;
+    float *w, *S;
     size_t bytes;
 };
 
-size_t score_ws_bytes(const abattn_dims *d, const abattn_params *p) {
-    const int64_t nqb = cdiv(d->N, 128), nkvb = cdiv(d->N, p->kv_block);
-    const int64_t crow = d->B * d->H * nqb * p->n_clusters;
-    const int64_t ntiles = cdiv(nkvb, SC_TN);
-    return align256(sizeof(float2) * crow * ntiles) + align256(sizeof(float2) * crow);
-}
-
 PlanWs carve(void *ws, const abattn_dims *d, const abattn_params *p) {
     const int64_t nqb = cdiv(d->N, 128), nkvb = cdiv(d->N, p->kv_block);
-    const int64_t BH = d->B * d->H, rows = BH * nqb, nc = p->n_clusters;
-    const int64_t crow = rows * nc, ntiles = cdiv(nkvb, SC_TN);
+    const int64_t BH = d->B * d->H, rows = BH * nqb;
     PlanWs w{};
     uint8_t *b = static_cast<uint8_t *>(ws);
     size_t off = 0;
@@ -128,14 +128,21 @@ PlanWs carve(void *ws, const abattn_dims *d, const abattn_params *p) {
         off += align256(n);
         return r;
     };
-    w.Kbar = reinterpret_cast<float *>(take(sizeof(float) * BH * nkvb * d->d));
-    w.C = reinterpret_cast<float *>(take(sizeof(float) * crow * d->d));
-    w.w = reinterpret_cast<float *>(take(sizeof(float) * crow));
+    w.Khi = reinterpret_cast<__nv_bfloat16 *>(take(2 * BH * nkvb * d->d));
+    w.Klo = reinterpret_cast<__nv_bfloat16 *>(take(2 * BH * nkvb * d->d));
+    w.Chi = reinterpret_cast<__nv_bfloat16 *>(take(2 * rows * 8 * d->d));
+    w.Clo = reinterpret_cast<__nv_bfloat16 *>(take(2 * rows * 8 * d->d));
+    w.w = reinterpret_cast<float *>(take(sizeof(float) * rows * p->n_clusters));
     w.S = reinterpret_cast<float *>(take(sizeof(float) * rows * nkvb));
-    w.partials = reinterpret_cast<float2 *>(take(sizeof(float2) * crow * ntiles));
-    w.stats = reinterpret_cast<float2 *>(take(sizeof(float2) * crow));
     w.bytes = off;
     return w;
+}
+
+// abattn_score workspace: the bf16 hi/lo operands made from the fp32 inputs.
+size_t score_ws_bytes(const abattn_dims *d, const abattn_params *p) {
+    const int64_t nqb = cdiv(d->N, 128), nkvb = cdiv(d->N, p->kv_block);
+    const int64_t BH = d->B * d->H, rows = BH * nqb;
+    return 2 * align256(2 * BH * nkvb * d->d) + 2 * align256(2 * rows * 8 * d->d);
 }
 
 int64_t capacity(int64_t nkvb, float budget) {
@@ -145,21 +152,22 @@ int64_t capacity(int64_t nkvb, float budget) {
 }
 
 // ---------------------------------------------------------------- launchers
-int launch_meanpool(const void *K, const abattn_dims *d, int kb, float *Kbar, cudaStream_t st) {
+int launch_meanpool(const void *K, const abattn_dims *d, int kb, float *Kbar, __nv_bfloat16 *Khi,
+                    __nv_bfloat16 *Klo, cudaStream_t st) {
     const int64_t nkvb = cdiv(d->N, kb), BH = d->B * d->H;
     const int64_t total = BH * nkvb * (d->d / 8);
     const int64_t want = cdiv(total, 256);
     const int grid = int(want < int64_t(sm_count()) * 32 ? want : int64_t(sm_count()) * 32);
     if (d->d == 128)
-        meanpool_kernel<128><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(K), BH, d->N, kb, nkvb, Kbar);
+        meanpool_kernel<128><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(K), BH, d->N, kb, nkvb, Kbar, Khi, Klo);
     else
-        meanpool_kernel<64><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(K), BH, d->N, kb, nkvb, Kbar);
+        meanpool_kernel<64><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(K), BH, d->N, kb, nkvb, Kbar, Khi, Klo);
     return launch_status();
 }
 
 template <int D>
 int launch_kmeans_t(const void *Q, const abattn_dims *d, const abattn_params *p, float *C, float *w,
-                    int32_t *labels, cudaStream_t st) {
+                    int32_t *labels, __nv_bfloat16 *Chi, __nv_bfloat16 *Clo, cudaStream_t st) {
     const int64_t nqb = cdiv(d->N, 128), rows = d->B * d->H * nqb;
     constexpr size_t smem = kmeans_smem_bytes<D>();
     static bool attr = false;
@@ -169,35 +177,44 @@ int launch_kmeans_t(const void *Q, const abattn_dims *d, const abattn_params *p,
         attr = true;
     }
     kmeans_kernel<D><<<unsigned(rows), KM_THREADS, smem, st>>>(
-        static_cast<const __nv_bfloat16 *>(Q), d->N, nqb, p->n_clusters, p->kmeans_iters, C, w, labels);
+        static_cast<const __nv_bfloat16 *>(Q), d->N, nqb, p->n_clusters, p->kmeans_iters, C, w, labels, Chi, Clo);
     return launch_status();
 }
 
 template <int D>
-int launch_score_t(const float *C, const float *w, const float *Kbar, const abattn_dims *d,
-                   const abattn_params *p, float *S, float2 *partials, float2 *stats, cudaStream_t st) {
+int launch_score_t(const __nv_bfloat16 *Chi, const __nv_bfloat16 *Clo, const __nv_bfloat16 *Khi,
+                   const __nv_bfloat16 *Klo, const float *w, const abattn_dims *d, const abattn_params *p,
+                   float *S, cudaStream_t st) {
     const int64_t nqb = cdiv(d->N, 128), nkvb = cdiv(d->N, p->kv_block), BH = d->B * d->H;
-    const int ntiles = int(cdiv(nkvb, SC_TN));
-    const float sl2 = resolve_scale(p->scale, d->d) * 1.4426950408889634f;
-    constexpr size_t smem = score_smem_bytes<D>();
+    CUtensorMap mChi, mClo, mKhi, mKlo;
+    int rc;
+    if ((rc = make_map_rows(&mChi, Chi, D, nqb * 8, BH, 128)) || (rc = make_map_rows(&mClo, Clo, D, nqb * 8, BH, 128)) ||
+        (rc = make_map_rows(&mKhi, Khi, D, nkvb, BH, 128)) || (rc = make_map_rows(&mKlo, Klo, D, nkvb, BH, 128)))
+        return rc;
+    ScoreParams sp;
+    sp.w = w;
+    sp.S = S;
+    sp.nqb = int(nqb);
+    sp.nkvb = int(nkvb);
+    sp.nc = p->n_clusters;
+    sp.scale_log2 = resolve_scale(p->scale, d->d) * 1.4426950408889634f;
+    constexpr int smem = ScoreLayout<D>::ALLOC;
     static bool attr = false;
     if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(score_pass1_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(score_pass2_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return cuda_status(e);
         attr = true;
     }
-    dim3 grid(unsigned(ntiles), unsigned(cdiv(nqb, SC_QB)), unsigned(BH));
-    score_pass1_kernel<D><<<grid, 256, smem, st>>>(C, Kbar, nqb, nkvb, p->n_clusters, sl2, partials, ntiles);
-    int rc = launch_status();
-    if (rc) return rc;
-    const int64_t crow = BH * nqb * p->n_clusters;
-    score_combine_kernel<<<unsigned(cdiv(crow, 256)), 256, 0, st>>>(partials, crow, ntiles, stats);
-    rc = launch_status();
-    if (rc) return rc;
-    score_pass2_kernel<D><<<grid, 256, smem, st>>>(C, w, Kbar, nqb, nkvb, p->n_clusters, sl2, stats, S);
+    dim3 grid(unsigned(cdiv(nqb, SC_QBT)), unsigned(BH));
+    score_tc_kernel<D><<<grid, SC_THREADS, smem, st>>>(mChi, mClo, mKhi, mKlo, sp);
     return launch_status();
+}
+
+int launch_score(const __nv_bfloat16 *Chi, const __nv_bfloat16 *Clo, const __nv_bfloat16 *Khi,
+                 const __nv_bfloat16 *Klo, const float *w, const abattn_dims *d, const abattn_params *p, float *S,
+                 cudaStream_t st) {
+    return d->d == 128 ? launch_score_t<128>(Chi, Clo, Khi, Klo, w, d, p, S, st)
+                       : launch_score_t<64>(Chi, Clo, Khi, Klo, w, d, p, S, st);
 }
 
 int launch_plan(int mode, const float *in, const abattn_dims *d, const abattn_params *p, int32_t *counts,
@@ -350,7 +367,7 @@ int abattn_meanpool(const void *K, const abattn_dims *dims, int32_t kv_block, fl
     if (K == nullptr || Kbar == nullptr) return ABATTN_ERR_NULL;
     if (!aligned16(K) || !aligned16(Kbar)) return ABATTN_ERR_ALIGN;
     if ((rc = check_device())) return rc;
-    return launch_meanpool(K, dims, kv_block, Kbar, static_cast<cudaStream_t>(stream));
+    return launch_meanpool(K, dims, kv_block, Kbar, nullptr, nullptr, static_cast<cudaStream_t>(stream));
 }
 
 int abattn_kmeans(const void *Q, const abattn_dims *dims, const abattn_params *p, float *C, float *w,
@@ -362,8 +379,8 @@ int abattn_kmeans(const void *Q, const abattn_dims *dims, const abattn_params *p
     if (!aligned16(Q)) return ABATTN_ERR_ALIGN;
     if ((rc = check_device())) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    return dims->d == 128 ? launch_kmeans_t<128>(Q, dims, p, C, w, labels, st)
-                          : launch_kmeans_t<64>(Q, dims, p, C, w, labels, st);
+    return dims->d == 128 ? launch_kmeans_t<128>(Q, dims, p, C, w, labels, nullptr, nullptr, st)
+                          : launch_kmeans_t<64>(Q, dims, p, C, w, labels, nullptr, nullptr, st);
 }
 
 int abattn_score(const float *C, const float *w, const float *Kbar, const abattn_dims *dims,
@@ -378,13 +395,24 @@ int abattn_score(const float *C, const float *w, const float *Kbar, const abattn
     if (!aligned16(ws)) return ABATTN_ERR_ALIGN;
     if ((rc = check_device())) return rc;
     const int64_t nqb = cdiv(dims->N, 128), nkvb = cdiv(dims->N, p->kv_block);
-    const int64_t crow = dims->B * dims->H * nqb * p->n_clusters;
-    float2 *partials = static_cast<float2 *>(ws);
-    float2 *stats = reinterpret_cast<float2 *>(static_cast<uint8_t *>(ws) +
-                                               align256(sizeof(float2) * crow * cdiv(nkvb, SC_TN)));
+    const int64_t BH = dims->B * dims->H, rows = BH * nqb;
+    uint8_t *b = static_cast<uint8_t *>(ws);
+    __nv_bfloat16 *Khi = reinterpret_cast<__nv_bfloat16 *>(b);
+    __nv_bfloat16 *Klo = reinterpret_cast<__nv_bfloat16 *>(b + align256(2 * BH * nkvb * dims->d));
+    __nv_bfloat16 *Chi = reinterpret_cast<__nv_bfloat16 *>(b + 2 * align256(2 * BH * nkvb * dims->d));
+    __nv_bfloat16 *Clo = reinterpret_cast<__nv_bfloat16 *>(b + 2 * align256(2 * BH * nkvb * dims->d) +
+                                                           align256(2 * rows * 8 * dims->d));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    return dims->d == 128 ? launch_score_t<128>(C, w, Kbar, dims, p, S, partials, stats, st)
-                          : launch_score_t<64>(C, w, Kbar, dims, p, S, partials, stats, st);
+    const int grid = sm_count() * 8;
+    if (dims->d == 128) {
+        split_rows_kernel<128><<<grid, 256, 0, st>>>(Kbar, BH * nkvb, 1, 1, Khi, Klo);
+        split_rows_kernel<128><<<grid, 256, 0, st>>>(C, rows, p->n_clusters, 8, Chi, Clo);
+    } else {
+        split_rows_kernel<64><<<grid, 256, 0, st>>>(Kbar, BH * nkvb, 1, 1, Khi, Klo);
+        split_rows_kernel<64><<<grid, 256, 0, st>>>(C, rows, p->n_clusters, 8, Chi, Clo);
+    }
+    if ((rc = launch_status())) return rc;
+    return launch_score(Chi, Clo, Khi, Klo, w, dims, p, S, st);
 }
 
 int abattn_plan_from_scores(const float *S, const abattn_dims *dims, const abattn_params *p, int32_t *counts,
@@ -428,13 +456,11 @@ int abattn_plan(const void *Q, const void *K, const abattn_dims *dims, const aba
     if (!aligned16(ws)) return ABATTN_ERR_ALIGN;
     if ((rc = check_device())) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if ((rc = launch_meanpool(K, dims, p->kv_block, w.Kbar, st))) return rc;
-    rc = dims->d == 128 ? launch_kmeans_t<128>(Q, dims, p, w.C, w.w, nullptr, st)
-                        : launch_kmeans_t<64>(Q, dims, p, w.C, w.w, nullptr, st);
+    if ((rc = launch_meanpool(K, dims, p->kv_block, nullptr, w.Khi, w.Klo, st))) return rc;
+    rc = dims->d == 128 ? launch_kmeans_t<128>(Q, dims, p, nullptr, w.w, nullptr, w.Chi, w.Clo, st)
+                        : launch_kmeans_t<64>(Q, dims, p, nullptr, w.w, nullptr, w.Chi, w.Clo, st);
     if (rc) return rc;
-    rc = dims->d == 128 ? launch_score_t<128>(w.C, w.w, w.Kbar, dims, p, w.S, w.partials, w.stats, st)
-                        : launch_score_t<64>(w.C, w.w, w.Kbar, dims, p, w.S, w.partials, w.stats, st);
-    if (rc) return rc;
+    if ((rc = launch_score(w.Chi, w.Clo, w.Khi, w.Klo, w.w, dims, p, w.S, st))) return rc;
     return launch_plan(p->mode == ABATTN_MODE_TOPK ? kPlanTopk : kPlanSip, w.S, dims, p, counts, idx, pi_sel,
                        cap, nullptr, st);
 }

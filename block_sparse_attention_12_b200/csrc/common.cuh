@@ -83,6 +83,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
     }
 }
 
+// Waits without looking at the abort flag (used to drain in-flight copies
+// before the CTA exits); bounded like mbar_wait.
+__device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity) {
+    long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (clock64() - t0 > kWaitLimitCycles) { raise_error(kErrTimeout); return; }
+    }
+}
+
 // ---------------------------------------------------------------- TMA
 // 3D tiled bulk-tensor load global -> shared, completion on an mbarrier.
 // Coordinates are (c0 innermost element, c1 row, c2 head).

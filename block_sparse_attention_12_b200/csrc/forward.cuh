@@ -70,15 +70,6 @@ struct FwdLayout {
     static constexpr int ALLOC = BYTES + 1024;  // slack for 1024-byte alignment
 };
 
-// Waits without looking at the abort flag (used to drain in-flight copies
-// before the CTA exits); bounded like mbar_wait.
-__device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity) {
-    long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
-        if (clock64() - t0 > kWaitLimitCycles) { raise_error(kErrTimeout); return; }
-    }
-}
-
 template <int HD, bool DENSE>
 __global__ void __launch_bounds__(FWD_THREADS, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,

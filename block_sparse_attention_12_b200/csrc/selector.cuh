@@ -13,11 +13,20 @@ namespace abattn {
 
 // ---------------------------------------------------------------- mean keys
 // One thread per (KV block, 8-column group): 16-byte bf16 loads, fp32 sums,
-// two 16-byte fp32 stores.  HBM bound: reads K once, writes Kbar once.
+// 16-byte stores.  HBM bound: reads K once, writes the mean keys once, either
+// as fp32 (Kbar) or as a bf16 pair hi + lo with hi = bf16(x), lo = bf16(x - hi)
+// (the operand format of the tensor-core score kernel), or both.
+__device__ __forceinline__ void split_bf16(float x, __nv_bfloat16 &hi, __nv_bfloat16 &lo) {
+    hi = __float2bfloat16_rn(x);
+    lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+}
+
 template <int D>
 __global__ void __launch_bounds__(256) meanpool_kernel(const __nv_bfloat16 *__restrict__ K,
                                                        int64_t BH, int64_t N, int kb,
-                                                       int64_t nkvb, float *__restrict__ Kbar) {
+                                                       int64_t nkvb, float *__restrict__ Kbar,
+                                                       __nv_bfloat16 *__restrict__ Khi,
+                                                       __nv_bfloat16 *__restrict__ Klo) {
     constexpr int G = D / 8;
     const int64_t total = BH * nkvb * G;
     for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
@@ -43,11 +52,38 @@ __global__ void __launch_bounds__(256) meanpool_kernel(const __nv_bfloat16 *__re
             }
         }
         const float cnt = float(t1 - t0);
-        float4 o0 = make_float4(acc[0] / cnt, acc[1] / cnt, acc[2] / cnt, acc[3] / cnt);
-        float4 o1 = make_float4(acc[4] / cnt, acc[5] / cnt, acc[6] / cnt, acc[7] / cnt);
-        float4 *dst = reinterpret_cast<float4 *>(Kbar + blk * D + c8 * 8);
-        dst[0] = o0;
-        dst[1] = o1;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) acc[u] = acc[u] / cnt;
+        if (Kbar != nullptr) {
+            float4 *dst = reinterpret_cast<float4 *>(Kbar + blk * D + c8 * 8);
+            dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+        }
+        if (Khi != nullptr) {
+            alignas(16) __nv_bfloat16 h[8], l[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) split_bf16(acc[u], h[u], l[u]);
+            *reinterpret_cast<uint4 *>(Khi + blk * D + c8 * 8) = *reinterpret_cast<const uint4 *>(h);
+            *reinterpret_cast<uint4 *>(Klo + blk * D + c8 * 8) = *reinterpret_cast<const uint4 *>(l);
+        }
+    }
+}
+
+// fp32 rows -> bf16 hi/lo pairs (used when the score stage gets fp32 inputs).
+// src rows of D floats, grouped n_in per block and padded to n_out rows per
+// block in the destination (the padding rows are zero).
+template <int D>
+__global__ void split_rows_kernel(const float *__restrict__ src, int64_t nblk, int n_in, int n_out,
+                                  __nv_bfloat16 *__restrict__ hi, __nv_bfloat16 *__restrict__ lo) {
+    const int64_t total = nblk * n_out * D;
+    for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
+         e += int64_t(gridDim.x) * blockDim.x) {
+        const int k = int(e % D);
+        const int64_t r = e / D;
+        const int c = int(r % n_out);
+        const int64_t b = r / n_out;
+        const float x = c < n_in ? src[(b * n_in + c) * D + k] : 0.f;
+        split_bf16(x, hi[e], lo[e]);
     }
 }
 
@@ -66,7 +102,8 @@ constexpr size_t kmeans_smem_bytes() {
 template <int D>
 __global__ void __launch_bounds__(KM_THREADS) kmeans_kernel(
     const __nv_bfloat16 *__restrict__ Q, int64_t N, int64_t nqb, int nc, int iters,
-    float *__restrict__ Cout, float *__restrict__ wout, int32_t *__restrict__ labels_out) {
+    float *__restrict__ Cout, float *__restrict__ wout, int32_t *__restrict__ labels_out,
+    __nv_bfloat16 *__restrict__ Chi, __nv_bfloat16 *__restrict__ Clo) {
     extern __shared__ float km_smem[];
     float *Qs = km_smem;                 // [D][KM_QS]
     float *Cs = Qs + D * KM_QS;          // [D][8]
@@ -163,159 +200,244 @@ __global__ void __launch_bounds__(KM_THREADS) kmeans_kernel(
     }
 
     const int64_t r = row;
-    for (int e = tid; e < nc * D; e += KM_THREADS) {
-        const int c = e / D, k = e % D;
-        Cout[(r * nc + c) * D + k] = Cs[k * 8 + c];
-    }
+    if (Cout != nullptr)
+        for (int e = tid; e < nc * D; e += KM_THREADS) {
+            const int c = e / D, k = e % D;
+            Cout[(r * nc + c) * D + k] = Cs[k * 8 + c];
+        }
+    if (Chi != nullptr)  // [rows][8][D], clusters past nc zero
+        for (int e = tid; e < 8 * D; e += KM_THREADS) {
+            const int c = e / D, k = e % D;
+            split_bf16(c < nc ? Cs[k * 8 + c] : 0.f, Chi[(r * 8 + c) * D + k], Clo[(r * 8 + c) * D + k]);
+        }
     if (tid < nc) wout[r * nc + tid] = iters > 0 ? float(cnt_s[tid]) / float(M) : 1.f / float(nc);
     if (labels_out != nullptr && tid < 128)
         labels_out[r * 128 + tid] = (iters > 0 && tid < M) ? lab[tid] : -1;
 }
 
 // ---------------------------------------------------------------- scores
-// Per head, the centroids of all q-blocks against all mean keys form a GEMM
-// [nqb*nc, d] x [d, nkvb].  A CTA computes a tile of 8 q-blocks (their nc <= 8
-// centroids each, 64 rows) x 128 KV blocks in fp32 on the CUDA cores: warp w
-// owns q-block w of the tile, lane l owns KV blocks l, l+32, l+64, l+96.
-// Pass 1 writes per-tile (max, sum exp) of every centroid row; a combine
-// kernel folds them into (m_c, Z_c); pass 2 recomputes the tile and writes
-// s_j = sum_c (w_c / Z_c) exp(L_cj - m_c).  Logits are kept in log2 units.
-constexpr int SC_QB = 8;
-constexpr int SC_TN = 128;
+// Per head, the centroids of all q-blocks against all mean keys form the GEMM
+// L = C Kbar^T ([nqb*8, d] x [d, nkvb]), evaluated on the tensor cores with
+// each fp32 operand split into a bf16 pair: C.K ~ Chi.Khi + Chi.Klo + Clo.Khi
+// (three kind::f16 MMAs into one fp32 TMEM accumulator; relative error about
+// 2^-16 of |C||K|).  One CTA owns 16 q-blocks (128 centroid rows) of one head
+// and sweeps the head's KV blocks twice:
+//   pass 1, rows = centroids: each epilogue thread owns one centroid row and
+//           keeps its running max m_c and normaliser Z_c = sum_j 2^(L_cj - m_c);
+//   pass 2, operands swapped, rows = KV blocks: each thread owns one KV block
+//           j and writes s_j = sum_c (w_c / Z_c) 2^(L_cj - m_c) for the 16
+//           q-blocks (the 8 clusters of a q-block are 8 columns of its row).
+// Warp 0 streams the Kbar tiles by TMA (2 stages), warp 1 issues the MMAs
+// into two TMEM accumulators, warps 2..5 run the epilogue.  Logits are in
+// log2 units.
+constexpr int SC_THREADS = 192;
+constexpr int SC_QBT = 16;  // q-blocks per CTA (x 8 cluster slots = 128 rows)
 
 template <int D>
-constexpr size_t score_smem_bytes() {
-    return sizeof(float) * size_t(SC_QB * 8 + SC_TN) * (D + 4);
-}
+struct ScoreLayout {
+    static constexpr int HALVES = D / 64;
+    static constexpr int TILE = HALVES * 16384;  // 128 rows x D bf16
+    static constexpr int C_HI = 0;
+    static constexpr int C_LO = TILE;
+    static constexpr int STAGE0 = 2 * TILE;  // stage s: hi at STAGE0 + 2*s*TILE, lo right after
+    static constexpr int MC_OFF = STAGE0 + 4 * TILE;
+    static constexpr int BAR_OFF = MC_OFF + 2 * 128 * 4;
+    static constexpr int NBARS = 9;
+    static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
+    static constexpr int BYTES = MISC_OFF + 16;
+    static constexpr int ALLOC = BYTES + 1024;
+};
+
+struct ScoreParams {
+    const float *w;  // [rows][nc]
+    float *S;        // [rows][nkvb]
+    int nqb;
+    int nkvb;
+    int nc;
+    float scale_log2;
+};
+
+__device__ __forceinline__ void epi_bar_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 template <int D>
-__device__ __forceinline__ void score_tile(const float *__restrict__ C, const float *__restrict__ Kbar,
-                                           int64_t bh, int64_t nqb, int64_t nkvb, int nc,
-                                           int64_t qb0, int64_t j0, float scale_log2,
-                                           float *smem, float (&L)[8][4]) {
-    constexpr int LD = D + 4;
-    float *Cs = smem;              // [64][LD]
-    float *Ks = smem + 64 * LD;    // [128][LD]
-    const int tid = threadIdx.x;
-    constexpr int V4 = D / 4;
-    for (int e = tid; e < 64 * V4; e += 256) {
-        const int r = e / V4, k4 = e % V4;
-        const int64_t qb = qb0 + r / 8;
-        const int c = r % 8;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (qb < nqb && c < nc)
-            v = __ldg(reinterpret_cast<const float4 *>(C + ((bh * nqb + qb) * nc + c) * D) + k4);
-        *reinterpret_cast<float4 *>(Cs + r * LD + 4 * k4) = v;
+__global__ void __launch_bounds__(SC_THREADS, 1)
+    score_tc_kernel(const __grid_constant__ CUtensorMap tmChi, const __grid_constant__ CUtensorMap tmClo,
+                    const __grid_constant__ CUtensorMap tmKhi, const __grid_constant__ CUtensorMap tmKlo,
+                    const ScoreParams p) {
+    using L = ScoreLayout<D>;
+    extern __shared__ uint8_t sc_smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(sc_smem_raw) + 1023) & ~uintptr_t(1023));
+    float *sm_m = reinterpret_cast<float *>(smem + L::MC_OFF);
+    float *sm_coef = sm_m + 128;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::BAR_OFF);
+    uint64_t *c_full = bars, *kv_full = bars + 1, *kv_empty = bars + 3, *acc_full = bars + 5,
+             *acc_free = bars + 7;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::MISC_OFF);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::MISC_OFF + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = blockIdx.x, bh = blockIdx.y;
+    const int NT = (p.nkvb + 127) / 128;
+    const int U = 2 * NT;  // tile visits over both passes
+
+    if (threadIdx.x == 0) {
+        mbar_init(c_full, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&kv_full[i], 1);
+            mbar_init(&kv_empty[i], 1);
+            mbar_init(&acc_full[i], 1);
+            mbar_init(&acc_free[i], 4);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
     }
-    for (int e = tid; e < SC_TN * V4; e += 256) {
-        const int r = e / V4, k4 = e % V4;
-        const int64_t j = j0 + r;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (j < nkvb) v = __ldg(reinterpret_cast<const float4 *>(Kbar + (bh * nkvb + j) * D) + k4);
-        *reinterpret_cast<float4 *>(Ks + r * LD + 4 * k4) = v;
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 256);
+        tmem_relinquish();
     }
+    tc_fence_before();
     __syncthreads();
-    const int w = tid >> 5, lane = tid & 31;
-    float acc[8][4];
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            mbar_arrive_expect_tx(c_full, 2 * L::TILE);
 #pragma unroll
-    for (int c = 0; c < 8; ++c)
+            for (int h = 0; h < L::HALVES; ++h) {
+                tma_load_3d(smem + L::C_HI + h * 16384, &tmChi, c_full, h * 64, g * 128, bh);
+                tma_load_3d(smem + L::C_LO + h * 16384, &tmClo, c_full, h * 64, g * 128, bh);
+            }
+            int issued = 0;
+            for (int u = 0; u < U; ++u) {
+                const int s = u & 1, t = u < NT ? u : u - NT;
+                if (u >= 2 && !mbar_wait(&kv_empty[s], ((u >> 1) - 1) & 1, abort_flag)) break;
+                uint8_t *dst = smem + L::STAGE0 + 2 * s * L::TILE;
+                mbar_arrive_expect_tx(&kv_full[s], 2 * L::TILE);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc[c][i] = 0.f;
-    const float *crow = Cs + (w * 8) * LD;
-#pragma unroll 2
-    for (int k = 0; k < D; k += 4) {
-        float4 kv[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) kv[i] = *reinterpret_cast<const float4 *>(Ks + (lane + 32 * i) * LD + k);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            const float4 cv = *reinterpret_cast<const float4 *>(crow + c * LD + k);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                acc[c][i] = fmaf(cv.x, kv[i].x, acc[c][i]);
-                acc[c][i] = fmaf(cv.y, kv[i].y, acc[c][i]);
-                acc[c][i] = fmaf(cv.z, kv[i].z, acc[c][i]);
-                acc[c][i] = fmaf(cv.w, kv[i].w, acc[c][i]);
+                for (int h = 0; h < L::HALVES; ++h) {
+                    tma_load_3d(dst + h * 16384, &tmKhi, &kv_full[s], h * 64, t * 128, bh);
+                    tma_load_3d(dst + L::TILE + h * 16384, &tmKlo, &kv_full[s], h * 64, t * 128, bh);
+                }
+                ++issued;
+            }
+            if (*abort_flag) {
+                mbar_drain(c_full, 0);
+                for (int u = issued - 2 < 0 ? 0 : issued - 2; u < issued; ++u) mbar_drain(&kv_full[u & 1], (u >> 1) & 1);
             }
         }
-    }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = make_idesc_bf16(128, 128, 0, 0);
+            const uint32_t cb = smem_u32(smem);
+            bool ok = mbar_wait(c_full, 0, abort_flag);
+            for (int u = 0; ok && u < U; ++u) {
+                const int s = u & 1, b = u & 1;
+                if (!mbar_wait(&kv_full[s], (u >> 1) & 1, abort_flag)) break;
+                if (u >= 2 && !mbar_wait(&acc_free[b], ((u >> 1) - 1) & 1, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t kb = cb + L::STAGE0 + 2 * s * L::TILE;
+                const uint32_t cbase = cb + L::C_HI;
+                // pass 1: A = centroids, B = mean keys; pass 2: swapped
+                const uint32_t a_hi = u < NT ? cbase : kb, a_lo = a_hi + L::TILE;
+                const uint32_t b_hi = u < NT ? kb : cbase, b_lo = b_hi + L::TILE;
+                const uint32_t dt = tmem + b * 128;
 #pragma unroll
-    for (int c = 0; c < 8; ++c)
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            L[c][i] = (j0 + lane + 32 * i < nkvb) ? acc[c][i] * scale_log2 : -INFINITY;
-}
-
-template <int D>
-__global__ void __launch_bounds__(256) score_pass1_kernel(
-    const float *__restrict__ C, const float *__restrict__ Kbar, int64_t nqb, int64_t nkvb, int nc,
-    float scale_log2, float2 *__restrict__ partials, int ntiles) {
-    extern __shared__ float sc_smem[];
-    const int64_t bh = blockIdx.z, qb0 = int64_t(blockIdx.y) * SC_QB, j0 = int64_t(blockIdx.x) * SC_TN;
-    float L[8][4];
-    score_tile<D>(C, Kbar, bh, nqb, nkvb, nc, qb0, j0, scale_log2, sc_smem, L);
-    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t qb = qb0 + w;
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        float m = fmaxf(fmaxf(L[c][0], L[c][1]), fmaxf(L[c][2], L[c][3]));
-        m = warp_max(m);
-        float z = 0.f;
-        if (m != -INFINITY) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) z += exp2f(L[c][i] - m);
-        }
-        z = warp_sum(z);
-        if (lane == 0 && qb < nqb && c < nc)
-            partials[((bh * nqb + qb) * nc + c) * ntiles + blockIdx.x] = make_float2(m, z);
-    }
-}
-
-// (m_c, Z_c) = fold of the per-tile partials, one thread per centroid row.
-__global__ void score_combine_kernel(const float2 *__restrict__ partials, int64_t nrows, int ntiles,
-                                     float2 *__restrict__ stats) {
-    const int64_t r = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (r >= nrows) return;
-    const float2 *p = partials + r * ntiles;
-    float m = -INFINITY;
-    for (int t = 0; t < ntiles; ++t) m = fmaxf(m, p[t].x);
-    float z = 0.f;
-    if (m != -INFINITY)
-        for (int t = 0; t < ntiles; ++t)
-            if (p[t].x != -INFINITY) z += p[t].y * exp2f(p[t].x - m);
-    stats[r] = make_float2(m, z);
-}
-
-template <int D>
-__global__ void __launch_bounds__(256) score_pass2_kernel(
-    const float *__restrict__ C, const float *__restrict__ w, const float *__restrict__ Kbar,
-    int64_t nqb, int64_t nkvb, int nc, float scale_log2, const float2 *__restrict__ stats,
-    float *__restrict__ S) {
-    extern __shared__ float sc_smem[];
-    const int64_t bh = blockIdx.z, qb0 = int64_t(blockIdx.y) * SC_QB, j0 = int64_t(blockIdx.x) * SC_TN;
-    float L[8][4];
-    score_tile<D>(C, Kbar, bh, nqb, nkvb, nc, qb0, j0, scale_log2, sc_smem, L);
-    const int wq = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t qb = qb0 + wq;
-    if (qb >= nqb) return;
-    const int64_t r = bh * nqb + qb;
-    float out[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        if (c < nc) {
-            const float2 st = stats[r * nc + c];
-            const float wc = __ldg(w + r * nc + c);
-            if (wc > 0.f && st.y > 0.f) {
-                const float coef = wc / st.y;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) out[i] = fmaf(coef, exp2f(L[c][i] - st.x), out[i]);
+                for (int k = 0; k < D / 16; ++k) {
+                    const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+                    umma_f16_ss(dt, make_sdesc_sw128(a_hi + off, 16, 1024), make_sdesc_sw128(b_hi + off, 16, 1024), idesc, k > 0);
+                    umma_f16_ss(dt, make_sdesc_sw128(a_hi + off, 16, 1024), make_sdesc_sw128(b_lo + off, 16, 1024), idesc, 1u);
+                    umma_f16_ss(dt, make_sdesc_sw128(a_lo + off, 16, 1024), make_sdesc_sw128(b_hi + off, 16, 1024), idesc, 1u);
+                }
+                umma_commit(&kv_empty[s]);
+                umma_commit(&acc_full[b]);
             }
         }
-    }
+        __syncwarp();
+    } else {
+        const int wq = warp & 3, rr = wq * 32 + lane;
+        const uint32_t t_lane = tmem + (uint32_t(wq * 32) << 16);
+        float m = -INFINITY, z = 0.f;
+        bool ok = true;
+        for (int u = 0; u < U; ++u) {
+            const int b = u & 1;
+            if (u == NT) {
+                // pass-1 statistics of this thread's centroid row -> shared memory
+                const int qb = g * SC_QBT + (rr >> 3), c = rr & 7;
+                float coef = 0.f;
+                if (qb < p.nqb && c < p.nc) {
+                    const float wc = p.w[(int64_t(bh) * p.nqb + qb) * p.nc + c];
+                    if (wc > 0.f && z > 0.f) coef = wc / z;
+                }
+                sm_m[rr] = m;
+                sm_coef[rr] = coef;
+                epi_bar_sync();
+            }
+            // on an abort every thread still runs all iterations (without
+            // work) so that all of them reach the named barrier above
+            if (!ok || !mbar_wait(&acc_full[b], (u >> 1) & 1, abort_flag)) { ok = false; continue; }
+            tc_fence_after();
+            uint32_t x[4][32];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int64_t j = j0 + lane + 32 * i;
-        if (j < nkvb) S[r * nkvb + j] = out[i];
+            for (int c = 0; c < 4; ++c) tmem_ld32(t_lane + b * 128 + c * 32, x[c]);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_free[b]);
+            if (u < NT) {
+                // pass 1: columns are KV blocks u*128 + col
+                const int j0 = u * 128;
+                float mt = -INFINITY;
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const float v = j0 + c * 32 + i < p.nkvb ? __uint_as_float(x[c][i]) * p.scale_log2 : -INFINITY;
+                        x[c][i] = __float_as_uint(v);
+                        mt = fmaxf(mt, v);
+                    }
+                const float mn = fmaxf(m, mt);
+                if (mn != -INFINITY) {
+                    float acc = 0.f;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) acc += exp2f(__uint_as_float(x[c][i]) - mn);
+                    z = z * exp2f(m - mn) + acc;
+                    m = mn;
+                }
+            } else {
+                // pass 2: this thread's row is KV block j; columns are centroid rows
+                const int j = (u - NT) * 128 + rr;
+#pragma unroll
+                for (int q = 0; q < SC_QBT; ++q) {
+                    const float4 m0 = *reinterpret_cast<const float4 *>(sm_m + q * 8);
+                    const float4 m1 = *reinterpret_cast<const float4 *>(sm_m + q * 8 + 4);
+                    const float4 k0 = *reinterpret_cast<const float4 *>(sm_coef + q * 8);
+                    const float4 k1 = *reinterpret_cast<const float4 *>(sm_coef + q * 8 + 4);
+                    const float mm[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+                    const float kk[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+                    float sv = 0.f;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const float lv = __uint_as_float(x[q >> 2][(q & 3) * 8 + c]) * p.scale_log2;
+                        if (kk[c] != 0.f) sv = fmaf(kk[c], exp2f(lv - mm[c]), sv);
+                    }
+                    const int qb = g * SC_QBT + q;
+                    if (j < p.nkvb && qb < p.nqb) p.S[(int64_t(bh) * p.nqb + qb) * p.nkvb + j] = sv;
+                }
+            }
+        }
+        (void)ok;
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
     }
 }
 
