@@ -266,7 +266,7 @@ int run_forward(bool dense, const void *Q, const void *K, const void *V, const a
     int rc = check_device();
     if (rc) return rc;
     CUtensorMap mQ, mK, mV;
-    const int box = dense ? 128 : kb;
+    const int box = dense ? 32 : (kb < 32 ? kb : 32);
     if ((rc = make_map(&mQ, Q, d, 128)) || (rc = make_map(&mK, K, d, box)) || (rc = make_map(&mV, V, d, box)))
         return rc;
     FwdParams fp;
@@ -279,6 +279,7 @@ int run_forward(bool dense, const void *Q, const void *K, const void *V, const a
     fp.N = int(d->N);
     fp.nqb = int(cdiv(d->N, 128));
     fp.kb = dense ? 128 : kb;
+    fp.box_rows = box;
     fp.nkvb = int(cdiv(d->N, fp.kb));
     fp.scale_log2 = resolve_scale(scale, d->d) * 1.4426950408889634f;
     const int64_t rows = d->B * d->H * fp.nqb;

@@ -8,24 +8,25 @@
 // paragraph: each selected block counts 1/pi times, realised as a shift of
 // the logits inside an ordinary softmax.
 //
-// One CTA per 128-query block, 192 threads, warp-specialised:
-//   warp 0      producer: TMA of the Q tile once; per 128-key tile, the
-//               selected KV blocks' K and V rows (one kb-row box per block and
-//               64-column half, 128-byte swizzle, 3 stages) and the tile's
-//               per-key log2(1/pi) bias into shared memory.  Each lane owns
-//               one block slot of the tile and fetches the plan entries of
-//               the next tile while the current one is in flight;
-//   warp 1      TMEM owner and MMA issuer: S = Q K^T (both operands in shared
-//               memory) into one of two TMEM buffers of 128 columns; O += P V
-//               with P read from TMEM (it overwrites the first 64 columns of
-//               its S buffer as packed bf16) and V from shared memory;
-//               tcgen05.commit to mbarriers;
-//   warps 2..5  softmax: one query row per thread (TMEM lane); logits
-//               t = s * scale * log2(e) + log2(1/pi); running max with lazy
-//               O rescaling (only when the max grows by more than 2^8);
-//               P = exp2(t - m) packed to bf16 and stored back to TMEM; the
-//               epilogue normalises O and writes O (bf16) and the
-//               natural-log LSE.
+// One CTA per 128-query block, 384 threads in three warpgroups:
+//   warps 0..3  softmax (setmaxnreg 240): one query row per thread (TMEM
+//               lane); logits t = s * scale * log2(e) + log2(1/pi); running
+//               max with lazy O rescaling (only when the max grows by more
+//               than 2^8); P = exp2(t - m) packed to bf16 and stored back to
+//               TMEM over the first 64 columns of its S buffer; the epilogue
+//               normalises O and writes O (bf16) and the natural-log LSE;
+//   warps 4..7  producers (setmaxnreg 64): warp 4 loads the Q tile once; warp
+//               4+w fills keys [32w, 32w+32) of every 128-key tile: for each
+//               selected KV block in that range, one TMA box of min(kb, 32)
+//               rows per 64-column half, for K and for V (128-byte swizzle,
+//               3 stages), plus those keys' log2(1/pi) bias.  Each lane owns
+//               one block slot and prefetches the next tile's plan entries.
+//               Small boxes cost the issuing warp tens of cycles each, so the
+//               128 boxes of a 4-token tile are spread over four warps;
+//   warp 8      TMEM owner and MMA issuer (warps 9..11 idle): S = Q K^T (both
+//               operands in shared memory) into one of two TMEM buffers of 128
+//               columns; O += P V with P read from TMEM and V from shared
+//               memory; tcgen05.commit to mbarriers.
 // The MMA warp issues QK^T of tile t+1 before PV of tile t, so the softmax
 // of one tile overlaps the tensor-core work of its neighbours; MMAs issued
 // by one thread run in order, so QK^T of tile t+2 cannot overwrite P(t)
@@ -36,7 +37,8 @@
 
 namespace abattn {
 
-constexpr int FWD_THREADS = 192;
+constexpr int FWD_THREADS = 384;
+constexpr int FWD_PRODUCERS = 4;  // producer warps, 32 keys of each tile apiece
 constexpr int FWD_NS = 3;  // K/V stages
 constexpr uint32_t FWD_TMEM_COLS = 512;
 constexpr uint32_t FWD_TMEM_O = 256;  // O accumulator column offset
@@ -51,6 +53,7 @@ struct FwdParams {
     int N;
     int nqb;
     int kb;
+    int box_rows;  // rows per K/V TMA box: min(kb, 32), 32 for the dense kernel
     int nkvb;
     float scale_log2;
 };
@@ -110,7 +113,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
         for (int s = 0; s < FWD_NS; ++s) {
-            mbar_init(&kv_full[s], 1);
+            mbar_init(&kv_full[s], FWD_PRODUCERS);
             mbar_init(&kv_empty[s], 1);
         }
         for (int i = 0; i < 2; ++i) mbar_init(&s_full[i], 1);
@@ -119,7 +122,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 1) {
+    if (warp == 8) {
         tmem_alloc(tmem_slot, FWD_TMEM_COLS);
         tmem_relinquish();
     }
@@ -128,34 +131,38 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ producer
-        if (lane == 0) {
+    if (warp >= 4 && warp < 8) {
+        // ------------------------------------------------------------ producers
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 64;\n" ::: "memory");
+        const int pw = warp - 4;
+        if (lane == 0 && pw == 0) {
             prefetch_tensormap(&tmQ);
             prefetch_tensormap(&tmK);
             prefetch_tensormap(&tmV);
         }
         int issued = 0;
         if (T > 0) {
-            if (lane == 0) {
+            if (lane == 0 && pw == 0) {
                 mbar_arrive_expect_tx(q_full, 128 * HD * 2);
 #pragma unroll
                 for (int h = 0; h < L::HALVES; ++h) tma_load_3d(sQ + h * 16384, &tmQ, q_full, h * 64, q0, bh);
             }
             const int32_t *ridx = DENSE ? nullptr : p.idx + int64_t(row) * p.cap;
             const float *rpi = DENSE ? nullptr : p.pi_sel + int64_t(row) * p.cap;
-            const int spt = DENSE ? 1 : 128 / p.kb;  // KV blocks per 128-key tile (<= 32)
-            int fill_blk = 0;                       // a valid block to load into padding slots
+            const int R = p.box_rows;                  // rows per box
+            const int nsl = 32 / R;                     // boxes (block slots) of this warp per tile
+            const int spt = DENSE ? 1 : 128 / p.kb;     // block slots per tile
+            const int slot0 = DENSE ? 0 : (32 * pw) / p.kb;  // this warp's first slot in the tile
+            int fill_blk = 0;                           // a valid block to load into padding slots
             if (!DENSE) {
                 const int b0 = ridx[0];
                 fill_blk = (b0 >= 0 && b0 < p.nkvb) ? b0 : 0;
             }
-            // plan entries of this lane's slot in tile t (prefetched one tile ahead)
             auto fetch = [&](int t, int &blk, float &pi) {
-                const int slot = t * spt + lane;
+                const int slot = t * spt + slot0 + lane;
                 blk = -1;
                 pi = 0.f;
-                if (!DENSE && lane < spt && slot < cnt) {
+                if (!DENSE && lane < nsl && slot < cnt) {
                     blk = __ldg(ridx + slot);
                     pi = __ldg(rpi + slot);
                 }
@@ -167,50 +174,43 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                 const int s = t % FWD_NS;
                 fetch(t + 1, nxt_blk, nxt_pi);
                 if (t >= FWD_NS && !mbar_wait(&kv_empty[s], ((t / FWD_NS) - 1) & 1, abort_flag)) break;
-                // this lane's slot: valid block and its bias
+                // this lane's block slot: validity and bias
                 bool mine_ok = false;
                 float mine_b = -INFINITY;
-                if (!DENSE && lane < spt && t * spt + lane < cnt) {
+                if (!DENSE && lane < nsl && t * spt + slot0 + lane < cnt) {
                     mine_ok = cur_blk >= 0 && cur_blk < p.nkvb && cur_pi > 0.f;
                     if (mine_ok) mine_b = -log2f(cur_pi);
                     else raise_error(kErrBounds);
                 }
-                // bias of keys 4*lane .. 4*lane+3 (all in one block since kb >= 4)
-                float bv[4];
+                // bias of key 32*pw + lane of the tile
+                float bias;
                 if (DENSE) {
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) bv[i] = (t * 128 + lane * 4 + i < p.N) ? 0.f : -INFINITY;
+                    bias = (t * 128 + 32 * pw + lane < p.N) ? 0.f : -INFINITY;
                 } else {
-                    const int owner = (lane * 4) / p.kb;
+                    const int owner = lane / R;
                     const float b = __shfl_sync(0xffffffffu, mine_b, owner);
                     const int blk = __shfl_sync(0xffffffffu, cur_blk, owner);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int key = blk * p.kb + (lane * 4 + i) % p.kb;
-                        bv[i] = key < p.N ? b : -INFINITY;
-                    }
+                    const int key = blk * p.kb + (32 * pw + lane) % p.kb;
+                    bias = key < p.N ? b : -INFINITY;
                 }
-                *reinterpret_cast<float4 *>(sBias + s * 128 + lane * 4) = make_float4(bv[0], bv[1], bv[2], bv[3]);
+                sBias[s * 128 + 32 * pw + lane] = bias;
                 __syncwarp();
-                if (lane == 0) mbar_arrive_expect_tx(&kv_full[s], 2 * 128 * HD * 2);
+                if (lane == 0) mbar_arrive_expect_tx(&kv_full[s], 32 * HD * 2 * 2);
                 __syncwarp();
                 uint8_t *dK = sK + s * L::TILE;
                 uint8_t *dV = sV + s * L::TILE;
-                if (DENSE) {
-                    if (lane == 0) {
-#pragma unroll
-                        for (int h = 0; h < L::HALVES; ++h) {
-                            tma_load_3d(dK + h * 16384, &tmK, &kv_full[s], h * 64, t * 128, bh);
-                            tma_load_3d(dV + h * 16384, &tmV, &kv_full[s], h * 64, t * 128, bh);
-                        }
+                if (lane < nsl) {
+                    const int drow = 32 * pw + lane * R;  // destination row in the tile
+                    int r0;
+                    if (DENSE) {
+                        r0 = t * 128 + drow;
+                    } else {
+                        r0 = (mine_ok ? cur_blk : fill_blk) * p.kb + drow % p.kb;
                     }
-                } else if (lane < spt) {
-                    const int r0 = (mine_ok ? cur_blk : fill_blk) * p.kb;
-                    const int off = lane * p.kb * 128;  // kb rows of 128 bytes per half
 #pragma unroll
                     for (int h = 0; h < L::HALVES; ++h) {
-                        tma_load_3d(dK + h * 16384 + off, &tmK, &kv_full[s], h * 64, r0, bh);
-                        tma_load_3d(dV + h * 16384 + off, &tmV, &kv_full[s], h * 64, r0, bh);
+                        tma_load_3d(dK + h * 16384 + drow * 128, &tmK, &kv_full[s], h * 64, r0, bh);
+                        tma_load_3d(dV + h * 16384 + drow * 128, &tmV, &kv_full[s], h * 64, r0, bh);
                     }
                 }
                 cur_blk = nxt_blk;
@@ -220,15 +220,16 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
             // drain: every issued copy lands before the CTA may exit
             if (*abort_flag) {
                 if (lane == 0) {
-                    mbar_drain(q_full, 0);
+                    if (pw == 0) mbar_drain(q_full, 0);
                     for (int t = issued - FWD_NS < 0 ? 0 : issued - FWD_NS; t < issued; ++t)
                         mbar_drain(&kv_full[t % FWD_NS], (t / FWD_NS) & 1);
                 }
             }
         }
-    } else if (warp == 1) {
+    } else if (warp >= 8) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0 && T > 0) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 64;\n" ::: "memory");
+        if (warp == 8 && lane == 0 && T > 0) {
             constexpr uint32_t idesc_qk = make_idesc_bf16(128, 128, 0, 0);
             constexpr uint32_t idesc_pv = make_idesc_bf16(128, HD, 0, 1);
             const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
@@ -268,6 +269,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------------------ softmax
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 240;\n" ::: "memory");
         const int wq = warp & 3;
         const int rr = wq * 32 + lane;
         const uint32_t t_lane = tmem + (uint32_t(wq * 32) << 16);
@@ -393,7 +395,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == 8) {
         tc_fence_after();
         tmem_dealloc(tmem, FWD_TMEM_COLS);
     }
