@@ -88,15 +88,23 @@ __global__ void split_rows_kernel(const float *__restrict__ src, int64_t nblk, i
 }
 
 // ---------------------------------------------------------------- k-means
-// One CTA (256 threads) per q-block.  The block's queries sit in shared
-// memory transposed, Qs[k][i] (row stride 129 floats: conflict-free column
-// and row walks); centroids interleaved, Cs[k][8].
-constexpr int KM_THREADS = 256;
-constexpr int KM_QS = 129;
+// One CTA (128 threads) per q-block.  The block's queries sit in shared
+// memory transposed and in their own bf16 precision, Qs[k][i] (row stride
+// 130 bf16: conflict-free column and row walks); centroids fp32,
+// interleaved, Cs[k][8].
+//   assignment: thread i scores its query against all 8 centroids as
+//               |c|^2 - 2 q.c (the same argmin as |q - c|^2; |q|^2 is
+//               common), ties to the lower index;
+//   update:     a stable counting sort of the labels (warp ballots) gives
+//               each cluster's members in ascending query order; thread k
+//               sums column k over each cluster's members.
+constexpr int KM_THREADS = 128;
+constexpr int KM_QS = 130;  // bf16 elements per Qs row (65 words: odd stride)
 
 template <int D>
 constexpr size_t kmeans_smem_bytes() {
-    return sizeof(float) * (size_t(D) * KM_QS + size_t(D) * 8 + 128 * 9) + sizeof(int) * (128 + 8);
+    return sizeof(__nv_bfloat16) * size_t(D) * KM_QS + sizeof(float) * (size_t(D) * 8 + 8 + 4 * 8) +
+           sizeof(int) * (128 + 128 + 8 + 9 + 4 * 8);
 }
 
 template <int D>
@@ -105,98 +113,138 @@ __global__ void __launch_bounds__(KM_THREADS) kmeans_kernel(
     float *__restrict__ Cout, float *__restrict__ wout, int32_t *__restrict__ labels_out,
     __nv_bfloat16 *__restrict__ Chi, __nv_bfloat16 *__restrict__ Clo) {
     extern __shared__ float km_smem[];
-    float *Qs = km_smem;                 // [D][KM_QS]
-    float *Cs = Qs + D * KM_QS;          // [D][8]
-    float *dist = Cs + D * 8;            // [128][9]
-    int *lab = reinterpret_cast<int *>(dist + 128 * 9);  // [128]
-    int *cnt_s = lab + 128;                               // [8]
+    __nv_bfloat16 *Qs = reinterpret_cast<__nv_bfloat16 *>(km_smem);               // [D][KM_QS]
+    float *Cs = km_smem + (D * KM_QS) / 2;                                         // [D][8]
+    float *cn = Cs + D * 8;                       // [8]     |c|^2
+    float *cn_part = cn + 8;                      // [4][8]  per-warp partial |c|^2
+    int *lab = reinterpret_cast<int *>(cn_part + 32);  // [128]
+    int *order = lab + 128;                        // [128]   queries sorted by cluster
+    int *cnt_s = order + 128;                      // [8]
+    int *start = cnt_s + 8;                        // [9]
+    int *wcnt = start + 9;                         // [4][8]  per-warp cluster counts
 
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int64_t row = blockIdx.x;
     const int64_t bh = row / nqb, qb = row % nqb;
     const int64_t q0 = qb * 128;
     const int M = int(N - q0 < 128 ? N - q0 : 128);
 
-    // load + transpose (bf16 -> fp32)
+    // load (all 16-byte loads in flight first) + transpose
     constexpr int G = D / 8;
+    constexpr int PER = (128 * G) / KM_THREADS;  // 16-byte chunks per thread
     const __nv_bfloat16 *src = Q + (bh * N + q0) * D;
-    for (int e = tid; e < M * G; e += KM_THREADS) {
-        const int i = e / G, c8 = e % G;
-        uint4 v = __ldg(reinterpret_cast<const uint4 *>(src + size_t(i) * D + c8 * 8));
-        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&v);
+    {
+        uint4 v[PER];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            float2 f = __bfloat1622float2(h[u]);
-            Qs[(c8 * 8 + 2 * u) * KM_QS + i] = f.x;
-            Qs[(c8 * 8 + 2 * u + 1) * KM_QS + i] = f.y;
+        for (int u = 0; u < PER; ++u) {
+            const int e = tid + u * KM_THREADS, i = e / G, c8 = e % G;
+            v[u] = i < M ? __ldg(reinterpret_cast<const uint4 *>(src + size_t(i) * D + c8 * 8)) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < PER; ++u) {
+            const int e = tid + u * KM_THREADS, i = e / G, c8 = e % G;
+            const __nv_bfloat16 *hv = reinterpret_cast<const __nv_bfloat16 *>(&v[u]);
+#pragma unroll
+            for (int x = 0; x < 8; ++x) Qs[(c8 * 8 + x) * KM_QS + i] = hv[x];
         }
     }
     __syncthreads();
     // init: centroid c = query floor(c*M/nc); unused centroid slots are zero
     for (int e = tid; e < D * 8; e += KM_THREADS) {
         const int k = e / 8, c = e % 8;
-        Cs[e] = c < nc ? Qs[k * KM_QS + (c * M) / nc] : 0.f;
+        Cs[e] = c < nc ? __bfloat162float(Qs[k * KM_QS + (c * M) / nc]) : 0.f;
     }
     if (tid < 8) cnt_s[tid] = 0;
     __syncthreads();
 
-    for (int it = 0; it < iters; ++it) {
-        // squared distances: thread -> (query i, centroids 4g .. 4g+3)
-        {
-            const int i = tid & 127, g = tid >> 7;
-            if (i < M && 4 * g < nc) {
-                float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll 8
-                for (int k = 0; k < D; ++k) {
-                    const float q = Qs[k * KM_QS + i];
-                    const float4 c = *reinterpret_cast<const float4 *>(Cs + k * 8 + 4 * g);
-                    float t;
-                    t = q - c.x; a0 = fmaf(t, t, a0);
-                    t = q - c.y; a1 = fmaf(t, t, a1);
-                    t = q - c.z; a2 = fmaf(t, t, a2);
-                    t = q - c.w; a3 = fmaf(t, t, a3);
-                }
-                dist[i * 9 + 4 * g + 0] = a0;
-                dist[i * 9 + 4 * g + 1] = a1;
-                dist[i * 9 + 4 * g + 2] = a2;
-                dist[i * 9 + 4 * g + 3] = a3;
-            }
+    auto centroid_norms = [&]() {
+        float part[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) part[c] = 0.f;
+        for (int k = tid; k < D; k += KM_THREADS) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) part[c] = fmaf(Cs[k * 8 + c], Cs[k * 8 + c], part[c]);
+        }
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const float v = warp_sum(part[c]);
+            if (lane == 0) cn_part[wid * 8 + c] = v;
         }
         __syncthreads();
+        if (tid < 8) cn[tid] = (cn_part[tid] + cn_part[8 + tid]) + (cn_part[16 + tid] + cn_part[24 + tid]);
+        __syncthreads();
+    };
+    if (iters > 0) centroid_norms();
+
+    for (int it = 0; it < iters; ++it) {
+        // assignment
+        int best = 0;
         if (tid < M) {
-            int best = 0;
-            float bd = dist[tid * 9];
-            for (int c = 1; c < nc; ++c) {
-                const float v = dist[tid * 9 + c];
-                if (v < bd) { bd = v; best = c; }
+            float a[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) a[c] = 0.f;
+#pragma unroll 4
+            for (int k = 0; k < D; ++k) {
+                const float q = __bfloat162float(Qs[k * KM_QS + tid]);
+                const float4 c0 = *reinterpret_cast<const float4 *>(Cs + k * 8);
+                const float4 c1 = *reinterpret_cast<const float4 *>(Cs + k * 8 + 4);
+                a[0] = fmaf(q, c0.x, a[0]);
+                a[1] = fmaf(q, c0.y, a[1]);
+                a[2] = fmaf(q, c0.z, a[2]);
+                a[3] = fmaf(q, c0.w, a[3]);
+                a[4] = fmaf(q, c1.x, a[4]);
+                a[5] = fmaf(q, c1.y, a[5]);
+                a[6] = fmaf(q, c1.z, a[6]);
+                a[7] = fmaf(q, c1.w, a[7]);
+            }
+            float bd = fmaf(-2.f, a[0], cn[0]);
+#pragma unroll
+            for (int c = 1; c < 8; ++c) {
+                const float v = fmaf(-2.f, a[c], cn[c]);
+                if (c < nc && v < bd) { bd = v; best = c; }
             }
             lab[tid] = best;
         }
+        // stable counting sort of the labels
+        unsigned my_rank = 0;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const unsigned m = __ballot_sync(0xffffffffu, tid < M && best == c);
+            if (best == c) my_rank = __popc(m & ((1u << lane) - 1u));
+            if (lane == 0) wcnt[wid * 8 + c] = __popc(m);
+        }
         __syncthreads();
-        // centroid update: thread -> (column k, CPT centroids)
-        {
-            constexpr int GROUPS = KM_THREADS / D;  // 2 for d=128, 4 for d=64
-            constexpr int CPT = 8 / GROUPS;
-            const int k = tid % D, grp = tid / D, c0 = grp * CPT;
-            float acc[CPT];
-            int n[CPT];
-#pragma unroll
-            for (int u = 0; u < CPT; ++u) { acc[u] = 0.f; n[u] = 0; }
-            for (int i = 0; i < M; ++i) {
-                const int l = lab[i];
-                const float v = Qs[k * KM_QS + i];
-#pragma unroll
-                for (int u = 0; u < CPT; ++u)
-                    if (l == c0 + u) { acc[u] += v; n[u] += 1; }
+        if (tid == 0) {
+            int acc = 0;
+            for (int c = 0; c < 8; ++c) {
+                start[c] = acc;
+                const int n = wcnt[c] + wcnt[8 + c] + wcnt[16 + c] + wcnt[24 + c];
+                cnt_s[c] = n;
+                acc += n;
             }
+            start[8] = acc;
+        }
+        __syncthreads();
+        if (tid < M) {
+            int pos = start[best] + int(my_rank);
+            for (int w = 0; w < wid; ++w) pos += wcnt[w * 8 + best];
+            order[pos] = tid;
+        }
+        __syncthreads();
+        // update: thread k sums column k over each cluster's members (ascending order)
+        for (int k = tid; k < D; k += KM_THREADS) {
 #pragma unroll
-            for (int u = 0; u < CPT; ++u) {
-                const int c = c0 + u;
-                if (c < nc && n[u] > 0) Cs[k * 8 + c] = acc[u] / float(n[u]);
-                if (k == 0 && c < 8) cnt_s[c] = n[u];
+            for (int c = 0; c < 8; ++c) {
+                const int n = cnt_s[c];
+                if (c < nc && n > 0) {
+                    float acc = 0.f;
+                    for (int p = start[c]; p < start[c + 1]; ++p) acc += __bfloat162float(Qs[k * KM_QS + order[p]]);
+                    Cs[k * 8 + c] = acc / float(n);
+                }
             }
         }
         __syncthreads();
+        if (it + 1 < iters) centroid_norms();
     }
 
     const int64_t r = row;
