@@ -8,40 +8,44 @@
 // paragraph: each selected block counts 1/pi times, realised as a shift of
 // the logits inside an ordinary softmax.
 //
-// One CTA per 128-query block, 384 threads in three warpgroups:
-//   warps 0..3  softmax (setmaxnreg 240): one query row per thread (TMEM
-//               lane); logits t = s * scale * log2(e) + log2(1/pi); running
-//               max with lazy O rescaling (only when the max grows by more
-//               than 2^8); P = exp2(t - m) packed to bf16 and stored back to
-//               TMEM over the first 64 columns of its S buffer; the epilogue
-//               normalises O and writes O (bf16) and the natural-log LSE;
-//   warps 4..7  producers (setmaxnreg 64): warp 4 loads the Q tile once; warp
-//               4+w fills keys [32w, 32w+32) of every 128-key tile: for each
+// One CTA per 128-query block, 512 threads in four warpgroups:
+//   warps 0..7  softmax, two warpgroups (setmaxnreg 208): warpgroup g takes
+//               the KV tiles t = g, g+2, g+4, ... with its own S buffer and
+//               its own O accumulator in TMEM, so the two run side by side
+//               and hide each other's latencies.  One query row per thread
+//               (TMEM lane); logits t = s * scale * log2(e) + log2(1/pi);
+//               running max with lazy O rescaling (only when the max grows by
+//               more than 2^8); P = exp2(t - m) packed to bf16 and stored back
+//               to TMEM over the first 64 columns of its S buffer.  At the end
+//               the two partial softmaxes are merged (max, sums, O) and O
+//               (bf16) and the natural-log LSE are written;
+//   warps 8..11 producers (setmaxnreg 40): warp 8 loads the Q tile once; warp
+//               8+w fills keys [32w, 32w+32) of every 128-key tile: for each
 //               selected KV block in that range, one TMA box of min(kb, 32)
 //               rows per 64-column half, for K and for V (128-byte swizzle,
 //               3 stages), plus those keys' log2(1/pi) bias.  Each lane owns
 //               one block slot and prefetches the next tile's plan entries.
 //               Small boxes cost the issuing warp tens of cycles each, so the
 //               128 boxes of a 4-token tile are spread over four warps;
-//   warp 8      TMEM owner and MMA issuer (warps 9..11 idle): S = Q K^T (both
-//               operands in shared memory) into one of two TMEM buffers of 128
-//               columns; O += P V with P read from TMEM and V from shared
+//   warp 12     TMEM owner and MMA issuer (warps 13..15 idle, setmaxnreg 40):
+//               S = Q K^T (both operands in shared memory) into S buffer
+//               t % 2; O_{t%2} += P V with P read from TMEM and V from shared
 //               memory; tcgen05.commit to mbarriers.
-// The MMA warp issues QK^T of tile t+1 before PV of tile t, so the softmax
-// of one tile overlaps the tensor-core work of its neighbours; MMAs issued
-// by one thread run in order, so QK^T of tile t+2 cannot overwrite P(t)
-// before PV(t) has read it.
+// TMEM: S0 [0,128), S1 [128,256), O_even [256,256+d), O_odd [384,384+d).
+// The MMA warp issues QK^T of tile t+1 before PV of tile t; MMAs issued by
+// one thread run in order, so QK^T of tile t+2 cannot overwrite P(t) before
+// PV(t) has read it.
 #pragma once
 
 #include "common.cuh"
 
 namespace abattn {
 
-constexpr int FWD_THREADS = 384;
+constexpr int FWD_THREADS = 512;
 constexpr int FWD_PRODUCERS = 4;  // producer warps, 32 keys of each tile apiece
 constexpr int FWD_NS = 3;  // K/V stages
 constexpr uint32_t FWD_TMEM_COLS = 512;
-constexpr uint32_t FWD_TMEM_O = 256;  // O accumulator column offset
+constexpr uint32_t FWD_TMEM_O = 256;  // O accumulators: even tiles at 256, odd tiles at 384
 
 struct FwdParams {
     const int32_t *counts;
@@ -67,7 +71,11 @@ struct FwdLayout {
     static constexpr int V_OFF = K_OFF + FWD_NS * TILE;
     static constexpr int BIAS_OFF = V_OFF + FWD_NS * TILE;
     static constexpr int BAR_OFF = BIAS_OFF + FWD_NS * 128 * 4;
-    static constexpr int NBARS = 1 + 2 * FWD_NS + 4;
+    static constexpr int NBARS = 1 + 2 * FWD_NS + 6;
+    // (m, l) of both softmax warpgroups, [2][2][128] floats, exchanged in the
+    // epilogue through the first K stage: by then every QK^T MMA has completed
+    // and every K load has landed
+    static constexpr int XCH_OFF = K_OFF;
     static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
     static constexpr int BYTES = MISC_OFF + 16;
     static constexpr int ALLOC = BYTES + 1024;  // slack for 1024-byte alignment
@@ -89,9 +97,10 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
     uint64_t *q_full = bars;
     uint64_t *kv_full = bars + 1;
     uint64_t *kv_empty = bars + 1 + FWD_NS;
-    uint64_t *s_full = bars + 1 + 2 * FWD_NS;
-    uint64_t *p_full = s_full + 2;
-    uint64_t *pv_done = p_full + 1;
+    uint64_t *s_full = bars + 1 + 2 * FWD_NS;  // [2]
+    uint64_t *p_full = s_full + 2;              // [2]
+    uint64_t *pv_done = p_full + 2;             // [2]
+    float *xch = reinterpret_cast<float *>(smem + L::XCH_OFF);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::MISC_OFF);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::MISC_OFF + 4);
 
@@ -116,13 +125,15 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
             mbar_init(&kv_full[s], FWD_PRODUCERS);
             mbar_init(&kv_empty[s], 1);
         }
-        for (int i = 0; i < 2; ++i) mbar_init(&s_full[i], 1);
-        mbar_init(p_full, 4);
-        mbar_init(pv_done, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s_full[i], 1);
+            mbar_init(&p_full[i], 4);
+            mbar_init(&pv_done[i], 1);
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 8) {
+    if (warp == 12) {
         tmem_alloc(tmem_slot, FWD_TMEM_COLS);
         tmem_relinquish();
     }
@@ -131,10 +142,10 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp >= 4 && warp < 8) {
+    if (warp >= 8 && warp < 12) {
         // ------------------------------------------------------------ producers
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 64;\n" ::: "memory");
-        const int pw = warp - 4;
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 40;\n" ::: "memory");
+        const int pw = warp - 8;
         if (lane == 0 && pw == 0) {
             prefetch_tensormap(&tmQ);
             prefetch_tensormap(&tmK);
@@ -226,10 +237,10 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                 }
             }
         }
-    } else if (warp >= 8) {
+    } else if (warp >= 12) {
         // ------------------------------------------------------------ MMA issuer
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 64;\n" ::: "memory");
-        if (warp == 8 && lane == 0 && T > 0) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 40;\n" ::: "memory");
+        if (warp == 12 && lane == 0 && T > 0) {
             constexpr uint32_t idesc_qk = make_idesc_bf16(128, 128, 0, 0);
             constexpr uint32_t idesc_pv = make_idesc_bf16(128, HD, 0, 1);
             const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
@@ -251,33 +262,38 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
             if (ok) ok = issue_qk(0);
             for (int t = 0; ok && t < T; ++t) {
                 if (t + 1 < T && !issue_qk(t + 1)) break;
-                if (!mbar_wait(p_full, t & 1, abort_flag)) break;
+                const int g = t & 1;  // softmax warpgroup / S buffer / O accumulator of this tile
+                if (!mbar_wait(&p_full[g], (t >> 1) & 1, abort_flag)) break;
                 tc_fence_after();
                 const int s = t % FWD_NS;
                 const uint32_t vbase = aV + s * L::TILE;
-                const uint32_t pbase = tmem + (t & 1) * 128;
+                const uint32_t pbase = tmem + g * 128;
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
-                    umma_f16_ts(tmem + FWD_TMEM_O, pbase + k * 8,
+                    umma_f16_ts(tmem + FWD_TMEM_O + g * 128, pbase + k * 8,
                                 make_sdesc_sw128(vbase + k * 2048, 16384, 1024), idesc_pv,
-                                (t > 0 || k > 0) ? 1u : 0u);
+                                (t >= 2 || k > 0) ? 1u : 0u);
                 }
                 umma_commit(&kv_empty[s]);
-                umma_commit(pv_done);
+                umma_commit(&pv_done[g]);
             }
         }
         __syncwarp();
     } else {
         // ------------------------------------------------------------ softmax
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 240;\n" ::: "memory");
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 208;\n" ::: "memory");
+        const int g = warp >> 2;  // 0: even tiles, 1: odd tiles
         const int wq = warp & 3;
         const int rr = wq * 32 + lane;
         const uint32_t t_lane = tmem + (uint32_t(wq * 32) << 16);
+        const uint32_t t_S = t_lane + g * 128;
+        const uint32_t t_O = t_lane + FWD_TMEM_O + g * 128;
         float m = -INFINITY, l = 0.f;
         bool ok = true;
-        for (int t = 0; t < T; ++t) {
-            const int s = t % FWD_NS, sb = t & 1;
-            if (!mbar_wait(&s_full[sb], (t >> 1) & 1, abort_flag) ||
+        int ntiles = 0;
+        for (int t = g; t < T; t += 2, ++ntiles) {
+            const int s = t % FWD_NS;
+            if (!mbar_wait(&s_full[g], (t >> 1) & 1, abort_flag) ||
                 !mbar_wait(&kv_full[s], (t / FWD_NS) & 1, abort_flag)) {
                 ok = false;
                 break;
@@ -285,60 +301,62 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
             tc_fence_after();
             uint32_t x[4][32];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(t_lane + sb * 128 + c * 32, x[c]);
+            for (int c = 0; c < 4; ++c) tmem_ld32(t_S + c * 32, x[c]);
             tmem_wait_ld();
 
             const float *bias = sBias + s * 128;
-            float mt = -INFINITY;
+            float mt0 = -INFINITY, mt1 = -INFINITY;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
 #pragma unroll
                 for (int i = 0; i < 32; i += 4) {
                     const float4 bb = *reinterpret_cast<const float4 *>(bias + c * 32 + i);
-                    float v0 = fmaf(__uint_as_float(x[c][i + 0]), p.scale_log2, bb.x);
-                    float v1 = fmaf(__uint_as_float(x[c][i + 1]), p.scale_log2, bb.y);
-                    float v2 = fmaf(__uint_as_float(x[c][i + 2]), p.scale_log2, bb.z);
-                    float v3 = fmaf(__uint_as_float(x[c][i + 3]), p.scale_log2, bb.w);
+                    const float v0 = fmaf(__uint_as_float(x[c][i + 0]), p.scale_log2, bb.x);
+                    const float v1 = fmaf(__uint_as_float(x[c][i + 1]), p.scale_log2, bb.y);
+                    const float v2 = fmaf(__uint_as_float(x[c][i + 2]), p.scale_log2, bb.z);
+                    const float v3 = fmaf(__uint_as_float(x[c][i + 3]), p.scale_log2, bb.w);
                     x[c][i + 0] = __float_as_uint(v0);
                     x[c][i + 1] = __float_as_uint(v1);
                     x[c][i + 2] = __float_as_uint(v2);
                     x[c][i + 3] = __float_as_uint(v3);
-                    mt = fmaxf(mt, fmaxf(fmaxf(v0, v1), fmaxf(v2, v3)));
+                    mt0 = fmaxf(mt0, fmaxf(v0, v1));
+                    mt1 = fmaxf(mt1, fmaxf(v2, v3));
                 }
             }
-            const float m_new = fmaxf(m, mt);
+            const float m_new = fmaxf(m, fmaxf(mt0, mt1));
             const bool need = m_new > m + 8.f;
             float alpha = 1.f;
             if (need) {
-                alpha = exp2f(m - m_new);
+                alpha = fast_exp2(m - m_new);
                 l *= alpha;
                 m = m_new;
             }
             const bool any = __any_sync(0xffffffffu, need);
             const float m_use = (m == -INFINITY) ? 0.f : m;
-            float rs = 0.f;
+            float rs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const float e = exp2f(__uint_as_float(x[c][i]) - m_use);
-                    rs += e;
+                    const float e = fast_exp2(__uint_as_float(x[c][i]) - m_use);
+                    rs[i & 3] += e;
                     x[c][i] = __float_as_uint(e);
                 }
             }
-            l += rs;
-            if (t > 0) {
-                if (!mbar_wait(pv_done, (t - 1) & 1, abort_flag)) { ok = false; break; }
+            l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+            if (ntiles > 0) {
+                // this warpgroup's O must be complete before it is rescaled
+                if (!mbar_wait(&pv_done[g], ((t >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 if (any) {
 #pragma unroll
                     for (int c = 0; c < HD / 32; ++c) {
                         uint32_t o[32];
-                        tmem_ld32(t_lane + FWD_TMEM_O + c * 32, o);
+                        tmem_ld32(t_O + c * 32, o);
                         tmem_wait_ld();
 #pragma unroll
                         for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                        tmem_st32(t_lane + FWD_TMEM_O + c * 32, o);
+                        tmem_st32(t_O + c * 32, o);
                     }
                     tmem_wait_st();
                 }
@@ -352,50 +370,76 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                     pk[i] = pack_bf16x2(__uint_as_float(x[c][2 * i]), __uint_as_float(x[c][2 * i + 1]));
                     pk[16 + i] = pack_bf16x2(__uint_as_float(x[c + 1][2 * i]), __uint_as_float(x[c + 1][2 * i + 1]));
                 }
-                tmem_st32(t_lane + sb * 128 + c * 16, pk);
+                tmem_st32(t_S + c * 16, pk);
             }
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(p_full);
+            if (lane == 0) mbar_arrive(&p_full[g]);
         }
         // ------------------------------------------------------------ epilogue
+        // wait for this warpgroup's last PV, swap (m, l) with the other
+        // warpgroup, then each warpgroup merges and writes half of the columns
+        bool done = ok && ntiles > 0;
+        if (done) {
+            const int t_last = g + 2 * (ntiles - 1);
+            done = mbar_wait(&pv_done[g], (t_last >> 1) & 1, abort_flag);
+        } else if (ok && T > 0) {
+            // no tile of our own (T == 1): the exchange area is K stage 0, so
+            // wait until QK^T of tile 0 has read it
+            mbar_wait(&s_full[0], 0, abort_flag);
+        }
+        xch[(g * 2 + 0) * 128 + rr] = done ? m : -INFINITY;
+        xch[(g * 2 + 1) * 128 + rr] = done ? l : 0.f;
+        tc_fence_before();
+        named_bar_sync(1, 256);
+        tc_fence_after();
+        const float m0 = xch[0 * 128 + rr], l0 = xch[1 * 128 + rr];
+        const float m1 = xch[2 * 128 + rr], l1 = xch[3 * 128 + rr];
+        const bool has0 = m0 != -INFINITY, has1 = m1 != -INFINITY;
+        const float mm = fmaxf(m0, m1);
+        const float a0 = has0 ? fast_exp2(m0 - mm) : 0.f;
+        const float a1 = has1 ? fast_exp2(m1 - mm) : 0.f;
+        const float lt = l0 * a0 + l1 * a1;
+        const float inv = lt > 0.f ? 1.f / lt : 0.f;
+        const float s0 = a0 * inv, s1 = a1 * inv;
         const int M = min(128, p.N - q0);
         const bool write = rr < M;
         __nv_bfloat16 *orow = p.O + (int64_t(bh) * p.N + q0 + rr) * HD;
-        if (ok && T > 0 && mbar_wait(pv_done, (T - 1) & 1, abort_flag)) {
-            tc_fence_after();
-            const float inv = l > 0.f ? 1.f / l : 0.f;
+        const uint32_t o0 = t_lane + FWD_TMEM_O, o1 = t_lane + FWD_TMEM_O + 128;
+        // this warpgroup writes columns [g*HD/2, (g+1)*HD/2); an accumulator
+        // that no tile reached is never read
 #pragma unroll
-            for (int c = 0; c < HD / 32; ++c) {
-                uint32_t o[32];
-                tmem_ld32(t_lane + FWD_TMEM_O + c * 32, o);
-                tmem_wait_ld();
-                if (write) {
+        for (int c = 0; c < HD / 64; ++c) {
+            const int col = g * (HD / 2) + c * 32;
+            uint32_t va[32], vb[32];
+            if (has0) tmem_ld32(o0 + col, va);
+            if (has1) tmem_ld32(o1 + col, vb);
+            tmem_wait_ld();
+            if (write) {
 #pragma unroll
-                    for (int i = 0; i < 32; i += 8) {
-                        uint4 v;
-                        v.x = pack_bf16x2(__uint_as_float(o[i + 0]) * inv, __uint_as_float(o[i + 1]) * inv);
-                        v.y = pack_bf16x2(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
-                        v.z = pack_bf16x2(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
-                        v.w = pack_bf16x2(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
-                        *reinterpret_cast<uint4 *>(orow + c * 32 + i) = v;
-                    }
+                for (int i = 0; i < 32; i += 8) {
+                    float f[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        f[u] = (has0 ? __uint_as_float(va[i + u]) * s0 : 0.f) +
+                               (has1 ? __uint_as_float(vb[i + u]) * s1 : 0.f);
+                    uint4 v;
+                    v.x = pack_bf16x2(f[0], f[1]);
+                    v.y = pack_bf16x2(f[2], f[3]);
+                    v.z = pack_bf16x2(f[4], f[5]);
+                    v.w = pack_bf16x2(f[6], f[7]);
+                    *reinterpret_cast<uint4 *>(orow + col + i) = v;
                 }
             }
-            if (write && p.lse != nullptr)
-                p.lse[int64_t(bh) * p.N + q0 + rr] =
-                    l > 0.f ? (m + log2f(l)) * 0.69314718055994530942f : -INFINITY;
-        } else if (write && (T == 0 || !ok)) {
-#pragma unroll
-            for (int i = 0; i < HD; i += 8) *reinterpret_cast<uint4 *>(orow + i) = make_uint4(0, 0, 0, 0);
-            if (p.lse != nullptr) p.lse[int64_t(bh) * p.N + q0 + rr] = -INFINITY;
         }
+        if (g == 0 && write && p.lse != nullptr)
+            p.lse[int64_t(bh) * p.N + q0 + rr] = lt > 0.f ? (mm + log2f(lt)) * 0.69314718055994530942f : -INFINITY;
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 8) {
+    if (warp == 12) {
         tc_fence_after();
         tmem_dealloc(tmem, FWD_TMEM_COLS);
     }
