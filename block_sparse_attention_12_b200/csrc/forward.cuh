@@ -9,7 +9,7 @@
 // the logits inside an ordinary softmax.
 //
 // One CTA per 128-query block, 512 threads in four warpgroups:
-//   warps 0..7  softmax, two warpgroups (setmaxnreg 208): warpgroup g takes
+//   warps 0..7  softmax, two warpgroups (setmaxnreg raised): warpgroup g takes
 //               the KV tiles t = g, g+2, g+4, ... with its own S buffer and
 //               its own O accumulator in TMEM, so the two run side by side
 //               and hide each other's latencies.  One query row per thread
@@ -19,18 +19,19 @@
 //               to TMEM over the first 64 columns of its S buffer.  At the end
 //               the two partial softmaxes are merged (max, sums, O) and O
 //               (bf16) and the natural-log LSE are written;
-//   warps 8..11 producers (setmaxnreg 40): warp 8 loads the Q tile once; warp
-//               8+w fills keys [32w, 32w+32) of every 128-key tile: for each
-//               selected KV block in that range, one TMA box of min(kb, 32)
-//               rows per 64-column half, for K and for V (128-byte swizzle,
-//               3 stages), plus those keys' log2(1/pi) bias.  Each lane owns
-//               one block slot and prefetches the next tile's plan entries.
-//               Small boxes cost the issuing warp tens of cycles each, so the
-//               128 boxes of a 4-token tile are spread over four warps;
-//   warp 12     TMEM owner and MMA issuer (warps 13..15 idle, setmaxnreg 40):
-//               S = Q K^T (both operands in shared memory) into S buffer
-//               t % 2; O_{t%2} += P V with P read from TMEM and V from shared
-//               memory; tcgen05.commit to mbarriers.
+//   warps 8..11, 13..15  producers (setmaxnreg lowered): warp 8 loads the Q
+//               tile once; a 128-key tile is cut into units of R = min(kb, 32)
+//               keys and producer w (0..6) owns units w, w+7, ...: per unit
+//               one TMA box of R rows per 64-column half, for K and for V
+//               (128-byte swizzle, 3 stages), and the bias log2(1/pi) of its R
+//               keys.  Each lane owns one unit and prefetches the next tile's
+//               plan entries.  Small boxes cost the issuing warp tens of cycles
+//               each, so the 128 boxes of a 4-token tile are spread over seven
+//               warps;
+//   warp 12     TMEM owner and MMA issuer (setmaxnreg lowered): S = Q K^T
+//               (both operands in shared memory) into S buffer t % 2;
+//               O_{t%2} += P V with P read from TMEM and V from shared memory;
+//               tcgen05.commit to mbarriers.
 // TMEM: S0 [0,128), S1 [128,256), O_even [256,256+d), O_odd [384,384+d).
 // The MMA warp issues QK^T of tile t+1 before PV of tile t; MMAs issued by
 // one thread run in order, so QK^T of tile t+2 cannot overwrite P(t) before
@@ -42,7 +43,20 @@
 namespace abattn {
 
 constexpr int FWD_THREADS = 512;
-constexpr int FWD_PRODUCERS = 4;  // producer warps, 32 keys of each tile apiece
+// setmaxnreg split (per thread): two softmax warpgroups take FWD_SOFTMAX_REGS,
+// the producer and MMA warpgroups FWD_OTHER_REGS; 2*128*S + 2*128*O must not
+// exceed the 512 x 128 registers the CTA launches with.
+#ifndef ABATTN_FWD_SOFTMAX_REGS
+#define ABATTN_FWD_SOFTMAX_REGS 208
+#endif
+#ifndef ABATTN_FWD_OTHER_REGS
+#define ABATTN_FWD_OTHER_REGS 48
+#endif
+constexpr int FWD_SOFTMAX_REGS = ABATTN_FWD_SOFTMAX_REGS;
+constexpr int FWD_OTHER_REGS = ABATTN_FWD_OTHER_REGS;
+static_assert(2 * 128 * FWD_SOFTMAX_REGS + 2 * 128 * FWD_OTHER_REGS <= FWD_THREADS * 128,
+              "setmaxnreg split exceeds the launch register budget");
+constexpr int FWD_PRODUCERS = 7;  // producer warps (8..11, 13..15); warp w owns the tile's block slots = w mod 7
 constexpr int FWD_NS = 3;  // K/V stages
 constexpr uint32_t FWD_TMEM_COLS = 512;
 constexpr uint32_t FWD_TMEM_O = 256;  // O accumulators: even tiles at 256, odd tiles at 384
@@ -57,7 +71,7 @@ struct FwdParams {
     int N;
     int nqb;
     int kb;
-    int box_rows;  // rows per K/V TMA box: min(kb, 32), 32 for the dense kernel
+    int box_rows;  // rows per K/V TMA box: min(kb, 32)
     int nkvb;
     float scale_log2;
 };
@@ -142,10 +156,10 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp >= 8 && warp < 12) {
+    if (warp >= 8 && warp != 12) {
         // ------------------------------------------------------------ producers
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 40;\n" ::: "memory");
-        const int pw = warp - 8;
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(FWD_OTHER_REGS) : "memory");
+        const int pw = warp < 12 ? warp - 8 : warp - 9;  // 0..6
         if (lane == 0 && pw == 0) {
             prefetch_tensormap(&tmQ);
             prefetch_tensormap(&tmK);
@@ -160,22 +174,29 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
             }
             const int32_t *ridx = DENSE ? nullptr : p.idx + int64_t(row) * p.cap;
             const float *rpi = DENSE ? nullptr : p.pi_sel + int64_t(row) * p.cap;
-            const int R = p.box_rows;                  // rows per box
-            const int nsl = 32 / R;                     // boxes (block slots) of this warp per tile
-            const int spt = DENSE ? 1 : 128 / p.kb;     // block slots per tile
-            const int slot0 = DENSE ? 0 : (32 * pw) / p.kb;  // this warp's first slot in the tile
-            int fill_blk = 0;                           // a valid block to load into padding slots
+            const int kb = p.kb;                      // rows per block (128 for the dense kernel)
+            const int R = p.box_rows;                 // rows per TMA box: min(kb, 32)
+            const int spt = 128 / kb;                 // block slots per tile
+            const int nunits = 128 / R;               // boxes (units) per tile and tensor half
+            const int unit = pw + FWD_PRODUCERS * lane;  // this lane's unit in every tile
+            const bool owner = unit < nunits;
+            const int sl = owner ? (unit * R) / kb : 0;  // the unit's block slot in the tile
+            const int ro = (unit * R) % kb;           // the unit's first row inside its block
+            // units owned by this warp in a tile: those congruent to pw modulo FWD_PRODUCERS
+            const int nown = nunits > pw ? (nunits - pw + FWD_PRODUCERS - 1) / FWD_PRODUCERS : 0;
+            const uint32_t tx_bytes = uint32_t(nown) * R * HD * 2 * 2;
+            int fill_blk = 0;                         // a valid block to load into padding slots
             if (!DENSE) {
                 const int b0 = ridx[0];
                 fill_blk = (b0 >= 0 && b0 < p.nkvb) ? b0 : 0;
             }
             auto fetch = [&](int t, int &blk, float &pi) {
-                const int slot = t * spt + slot0 + lane;
+                const int e = t * spt + sl;
                 blk = -1;
                 pi = 0.f;
-                if (!DENSE && lane < nsl && slot < cnt) {
-                    blk = __ldg(ridx + slot);
-                    pi = __ldg(rpi + slot);
+                if (!DENSE && owner && e < cnt) {
+                    blk = __ldg(ridx + e);
+                    pi = __ldg(rpi + e);
                 }
             };
             int cur_blk, nxt_blk;
@@ -185,45 +206,49 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                 const int s = t % FWD_NS;
                 fetch(t + 1, nxt_blk, nxt_pi);
                 if (t >= FWD_NS && !mbar_wait(&kv_empty[s], ((t / FWD_NS) - 1) & 1, abort_flag)) break;
-                // this lane's block slot: validity and bias
-                bool mine_ok = false;
-                float mine_b = -INFINITY;
-                if (!DENSE && lane < nsl && t * spt + slot0 + lane < cnt) {
-                    mine_ok = cur_blk >= 0 && cur_blk < p.nkvb && cur_pi > 0.f;
-                    if (mine_ok) mine_b = -log2f(cur_pi);
-                    else raise_error(kErrBounds);
-                }
-                // bias of key 32*pw + lane of the tile
-                float bias;
-                if (DENSE) {
-                    bias = (t * 128 + 32 * pw + lane < p.N) ? 0.f : -INFINITY;
-                } else {
-                    const int owner = lane / R;
-                    const float b = __shfl_sync(0xffffffffu, mine_b, owner);
-                    const int blk = __shfl_sync(0xffffffffu, cur_blk, owner);
-                    const int key = blk * p.kb + (32 * pw + lane) % p.kb;
-                    bias = key < p.N ? b : -INFINITY;
-                }
-                sBias[s * 128 + 32 * pw + lane] = bias;
-                __syncwarp();
-                if (lane == 0) mbar_arrive_expect_tx(&kv_full[s], 32 * HD * 2 * 2);
-                __syncwarp();
-                uint8_t *dK = sK + s * L::TILE;
-                uint8_t *dV = sV + s * L::TILE;
-                if (lane < nsl) {
-                    const int drow = 32 * pw + lane * R;  // destination row in the tile
-                    int r0;
+                if (owner) {
+                    // block of this unit, its validity and the bias of its R keys
+                    int blk;
+                    float b = -INFINITY;
                     if (DENSE) {
-                        r0 = t * 128 + drow;
+                        blk = t;
+                        b = 0.f;
+                    } else if (t * spt + sl < cnt) {
+                        const bool ok_blk = cur_blk >= 0 && cur_blk < p.nkvb && cur_pi > 0.f;
+                        if (ok_blk) {
+                            blk = cur_blk;
+                            b = -log2f(cur_pi);
+                        } else {
+                            blk = fill_blk;
+                            if (ro == 0) raise_error(kErrBounds);
+                        }
                     } else {
-                        r0 = (mine_ok ? cur_blk : fill_blk) * p.kb + drow % p.kb;
+                        blk = fill_blk;  // padding slot: loaded, weighted zero
                     }
+                    const int key0 = blk * kb + ro;
+                    float *bdst = sBias + s * 128 + unit * R;
+                    for (int i = 0; i < R; i += 4) {
+                        float4 v;
+                        v.x = key0 + i + 0 < p.N ? b : -INFINITY;
+                        v.y = key0 + i + 1 < p.N ? b : -INFINITY;
+                        v.z = key0 + i + 2 < p.N ? b : -INFINITY;
+                        v.w = key0 + i + 3 < p.N ? b : -INFINITY;
+                        *reinterpret_cast<float4 *>(bdst + i) = v;
+                    }
+                    __syncwarp(__activemask());
+                    if (lane == 0) mbar_arrive_expect_tx(&kv_full[s], tx_bytes);
+                    __syncwarp(__activemask());
+                    uint8_t *dK = sK + s * L::TILE + unit * R * 128;
+                    uint8_t *dV = sV + s * L::TILE + unit * R * 128;
 #pragma unroll
                     for (int h = 0; h < L::HALVES; ++h) {
-                        tma_load_3d(dK + h * 16384 + drow * 128, &tmK, &kv_full[s], h * 64, r0, bh);
-                        tma_load_3d(dV + h * 16384 + drow * 128, &tmV, &kv_full[s], h * 64, r0, bh);
+                        tma_load_3d(dK + h * 16384, &tmK, &kv_full[s], h * 64, key0, bh);
+                        tma_load_3d(dV + h * 16384, &tmV, &kv_full[s], h * 64, key0, bh);
                     }
+                } else if (lane == 0) {
+                    mbar_arrive_expect_tx(&kv_full[s], 0);  // a warp without units still arrives
                 }
+                __syncwarp();
                 cur_blk = nxt_blk;
                 cur_pi = nxt_pi;
                 ++issued;
@@ -237,10 +262,10 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                 }
             }
         }
-    } else if (warp >= 12) {
+    } else if (warp == 12) {
         // ------------------------------------------------------------ MMA issuer
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 40;\n" ::: "memory");
-        if (warp == 12 && lane == 0 && T > 0) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(FWD_OTHER_REGS) : "memory");
+        if (lane == 0 && T > 0) {
             constexpr uint32_t idesc_qk = make_idesc_bf16(128, 128, 0, 0);
             constexpr uint32_t idesc_pv = make_idesc_bf16(128, HD, 0, 1);
             const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
@@ -281,7 +306,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------------------ softmax
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 208;\n" ::: "memory");
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(FWD_SOFTMAX_REGS) : "memory");
         const int g = warp >> 2;  // 0: even tiles, 1: odd tiles
         const int wq = warp & 3;
         const int rr = wq * 32 + lane;
@@ -344,8 +369,20 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                 }
             }
             l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+            // P row -> TMEM, packed bf16 pairs over the first 64 columns of this S buffer
+#pragma unroll
+            for (int c = 0; c < 4; c += 2) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    pk[i] = pack_bf16x2(__uint_as_float(x[c][2 * i]), __uint_as_float(x[c][2 * i + 1]));
+                    pk[16 + i] = pack_bf16x2(__uint_as_float(x[c + 1][2 * i]), __uint_as_float(x[c + 1][2 * i + 1]));
+                }
+                tmem_st32(t_S + c * 16, pk);
+            }
             if (ntiles > 0) {
-                // this warpgroup's O must be complete before it is rescaled
+                // this warpgroup's O must be complete before it is rescaled;
+                // PV(t) is issued only after p_full below
                 if (!mbar_wait(&pv_done[g], ((t >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 if (any) {
@@ -358,19 +395,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                         for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
                         tmem_st32(t_O + c * 32, o);
                     }
-                    tmem_wait_st();
                 }
-            }
-            // P row -> TMEM, packed bf16 pairs over the first 64 columns of this S buffer
-#pragma unroll
-            for (int c = 0; c < 4; c += 2) {
-                uint32_t pk[32];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    pk[i] = pack_bf16x2(__uint_as_float(x[c][2 * i]), __uint_as_float(x[c][2 * i + 1]));
-                    pk[16 + i] = pack_bf16x2(__uint_as_float(x[c + 1][2 * i]), __uint_as_float(x[c + 1][2 * i + 1]));
-                }
-                tmem_st32(t_S + c * 16, pk);
             }
             tmem_wait_st();
             tc_fence_before();
