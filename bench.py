@@ -57,6 +57,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="budget x kv_block x (SIP, top-k) sweep on the sweep-75k layer, one JSON line per point")
     return ap.parse_args()
 
 
@@ -247,8 +249,60 @@ def timed(fn, iters, stream):
     return e0.elapsed_time(e1) / iters
 
 
+def run_sweep(args):
+    """Budget 5/8/11/25/50/100% x kv_block 4/128 x (SIP, top-k) on the
+    75,600-token x 10-head layer: plan and forward time, executed TFLOP/s,
+    relative-L2 error of O against the in-house dense kernel, and the ratio
+    of the sparse to the dense softmax normaliser (top-k: the retained
+    attention mass; SIP: about 1, the Horvitz-Thompson normaliser being
+    unbiased)."""
+    from block_sparse_attention_12_b200 import abi, build
+    build.build()
+    torch.cuda.set_device(0)
+    w = inputs.SWEEP
+    Q, K, V = inputs.make_qkv(w, device="cuda")
+    shape = tuple(Q.shape)
+    stream = torch.cuda.current_stream()
+    Od = torch.empty_like(Q)
+    _, lse_d = abi.dense_forward(Q, K, V, O=Od)
+    dense_ms = timed(lambda: abi.dense_forward(Q, K, V, O=Od, want_lse=False), 3, stream)
+    dfl = 4.0 * w.B * w.H * w.N * w.N * w.d
+    print(json.dumps({"sweep": "dense", "workload": w.name, "ms": dense_ms, "tflops": dfl / dense_ms / 1e9}), flush=True)
+    O = torch.empty_like(Q)
+    lse = torch.empty(shape[:3], dtype=torch.float32, device="cuda")
+    odn = Od.float().norm()
+    for kb in (4, 128):
+        for budget in (0.05, 0.08, 0.11, 0.25, 0.5, 1.0):
+            for mode in (abi.MODE_SIP, abi.MODE_TOPK):
+                cfg = abi.Config(kv_block=kb, budget=budget, mode=mode, seed=w.seed)
+                planner = abi.Planner(shape, cfg)
+                plan = planner(Q, K)
+                abi.forward(Q, K, V, plan, cfg, O=O, lse=lse)
+                abi.check()
+                plan_ms = timed(lambda: planner(Q, K), 3, stream)
+                fwd_ms = timed(lambda: abi.forward(Q, K, V, plan, cfg, O=O, lse=lse), 5, stream)
+                abi.check()
+                efl = abi.executed_flops(plan, shape)
+                err = float((O.float() - Od.float()).norm() / odn)
+                ratio = torch.exp(lse.double() - lse_d.double())
+                nkvb = -(-w.N // kb)
+                print(json.dumps({
+                    "sweep": "point", "workload": w.name, "kv_block": kb, "budget": budget,
+                    "mode": "SIP" if mode == abi.MODE_SIP else "TOPK",
+                    "selected_blocks_mean": float(plan.counts.float().mean()), "nkvb": nkvb,
+                    "plan_ms": plan_ms, "fwd_ms": fwd_ms, "executed_tflops": efl / fwd_ms / 1e9,
+                    "fwd_vs_dense_speedup": dense_ms / fwd_ms, "rel_l2_vs_dense": err,
+                    "normaliser_ratio_mean": float(ratio.mean()), "normaliser_ratio_p05": float(ratio.quantile(0.05)) if ratio.numel() < 2**24 else None,
+                }), flush=True)
+                del planner, plan
+                torch.cuda.empty_cache()
+
+
 def main():
     args = parse()
+    if args.sweep:
+        run_sweep(args)
+        return
     w = inputs.WORKLOADS[args.workload]
     if args.heads:
         import dataclasses

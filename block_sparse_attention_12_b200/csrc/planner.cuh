@@ -46,16 +46,32 @@ __device__ __forceinline__ void philox4x64_10(uint64_t &x0, uint64_t &x1, uint64
     }
 }
 
-// Uniforms for blocks 4m .. 4m+3 of row (b, h, qb): counter (m, qb, h, b),
-// key (seed, 0); each 64-bit word gives its top 24 bits times 2^-24.
-__device__ __forceinline__ void row_uniforms(uint64_t seed, int64_t b, int64_t h, int64_t qb,
-                                             int64_t m, float (&u)[4]) {
-    uint64_t x0 = uint64_t(m), x1 = uint64_t(qb), x2 = uint64_t(h), x3 = uint64_t(b);
-    philox4x64_10(x0, x1, x2, x3, seed, 0ull);
-    u[0] = float(uint32_t(x0 >> 40)) * 5.9604644775390625e-8f;  // 2^-24
-    u[1] = float(uint32_t(x1 >> 40)) * 5.9604644775390625e-8f;
-    u[2] = float(uint32_t(x2 >> 40)) * 5.9604644775390625e-8f;
-    u[3] = float(uint32_t(x3 >> 40)) * 5.9604644775390625e-8f;
+// Uniforms for blocks 8m .. 8m+7 of row (b, h, qb): counter (m, qb, h, b),
+// key (seed, 0); 64-bit word i gives blocks 8m+2i (its high 32-bit half) and
+// 8m+2i+1 (its low half), each as the half's top 24 bits times 2^-24.
+__device__ __forceinline__ void row_uniforms8(uint64_t seed, int64_t b, int64_t h, int64_t qb,
+                                              int64_t m, float (&u)[8]) {
+    uint64_t x[4] = {uint64_t(m), uint64_t(qb), uint64_t(h), uint64_t(b)};
+    philox4x64_10(x[0], x[1], x[2], x[3], seed, 0ull);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        u[2 * i] = float(uint32_t(x[i] >> 40)) * 5.9604644775390625e-8f;                 // 2^-24
+        u[2 * i + 1] = float(uint32_t(x[i] & 0xFFFFFFFFull) >> 8) * 5.9604644775390625e-8f;
+    }
+}
+
+// vals[j0 .. j0+7] (zero past `end`); two 16-byte shared loads when the
+// eight lie inside the row (j0 is a multiple of 8, so they are aligned).
+__device__ __forceinline__ void load8(const float *vals, int64_t j0, int64_t end, float (&r)[8]) {
+    if (j0 + 8 <= end) {
+        const float4 a = *reinterpret_cast<const float4 *>(vals + j0);
+        const float4 b = *reinterpret_cast<const float4 *>(vals + j0 + 4);
+        r[0] = a.x; r[1] = a.y; r[2] = a.z; r[3] = a.w;
+        r[4] = b.x; r[5] = b.y; r[6] = b.z; r[7] = b.w;
+    } else {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) r[u] = j0 + u < end ? vals[j0 + u] : 0.f;
+    }
 }
 
 struct PlanScratch {
@@ -88,8 +104,10 @@ __device__ __forceinline__ T block_sum(T v, T *warp_buf, T *bcast) {
 
 // One CTA per q-block row.  The row's scores (or probabilities) sit in
 // shared memory; warp w owns the contiguous segment [seg*w, seg*(w+1)) of
-// blocks (seg a multiple of 128), so selections are compacted per warp with
-// ballots and only the per-warp counts need a block-wide prefix.
+// blocks (seg a multiple of 256) and each lane 8 consecutive blocks at a
+// time, whose flags (capped, then taken) form one byte of `flags`.  Sampled
+// indices are compacted per warp with shuffles; only the per-warp counts
+// need a block-wide exchange, so they come out in ascending order.
 template <int MODE>
 __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
     const float *__restrict__ in, int64_t H, int64_t nqb, int64_t nkvb, double Bblk, int64_t k_top,
@@ -98,12 +116,12 @@ __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
     extern __shared__ float pl_smem[];
     __shared__ PlanScratch sc;
     float *vals = pl_smem;                                                   // [nkvb]
-    uint32_t *bits = reinterpret_cast<uint32_t *>(vals + nkvb);              // [ceil(nkvb/32)] flags
+    uint8_t *flags = reinterpret_cast<uint8_t *>(vals + nkvb);               // [ceil(nkvb/32) words]
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int64_t row = blockIdx.x;
     const int64_t b = row / (H * nqb), h = (row / nqb) % H, qb = row % nqb;
     const float *src = in + row * nkvb;
-    const int nwords = int((nkvb + 31) / 32);
+    const int nbytes = int((nkvb + 31) / 32) * 4;
 
     // load (8 independent loads in flight per thread); SIP also counts
     // positive scores and sums them
@@ -128,48 +146,67 @@ __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
             }
         }
     }
-    for (int w = tid; w < nwords; w += PL_THREADS) bits[w] = 0u;  // SIP: capped flags
+    for (int i = tid; i < nbytes; i += PL_THREADS) flags[i] = 0;
+
+    // this warp's segment; lane works on blocks j0 .. j0+7 of each 256-block step
+    const int64_t seg = ((nkvb + PL_WARPS * 256 - 1) / (PL_WARPS * 256)) * 256;
+    const int64_t w0 = int64_t(wid) * seg;
+    const int64_t w1 = w0 + seg < nkvb ? w0 + seg : nkvb;
 
     if (MODE == kPlanSip) {
         const int npos = block_sum<int>(npos_l, sc.iwarp, &sc.bcast[0]);  // (also orders the loads)
         if (Bblk >= double(npos)) {
             for (int64_t j = tid; j < nkvb; j += PL_THREADS) vals[j] = vals[j] > 0.f ? 1.f : 0.f;
         } else {
-            // capping rounds: lambda = (Bblk - |C|) / sum_{j not in C} s_j; C grows by
-            // {j : lambda s_j >= 1}; each pass also sums the scores left uncapped
+            // capping rounds: lambda = (Bblk - |C|) / sum_{j not in C} s_j; C
+            // grows by {j : lambda s_j >= 1}, tested exactly in fp64 for the
+            // blocks an fp32 product puts near the threshold; the uncapped sum
+            // is updated by subtracting the newly capped scores.  Lane-strided
+            // walk (conflict-free shared loads); the capped flags of 32
+            // consecutive blocks form one word, rebuilt by ballot.
+            uint32_t *fw = reinterpret_cast<uint32_t *>(flags);
             double rest = block_sum<double>(sum_l, sc.dwarp, &sc.dbcast);
             int64_t ncap = 0;
-            double lam = (Bblk - double(ncap)) / rest;
+            double lam = Bblk / rest;
             for (int64_t round = 0; round <= nkvb; ++round) {
+                const float near = float(lam) * (1.f + 1e-5f);
                 int added_l = 0;
-                double rest_l = 0.0;
-                for (int64_t j = tid; j < nkvb; j += PL_THREADS) {
-                    const int w = int(j >> 5);
-                    const uint32_t bit = 1u << (j & 31);
-                    if (bits[w] & bit) continue;
-                    const double sv = double(vals[j]);
-                    if (lam * sv >= 1.0) {
-                        atomicOr(&bits[w], bit);
-                        ++added_l;
-                    } else {
-                        rest_l += sv;
+                double capped_l = 0.0;
+                for (int64_t j32 = w0; j32 < w1; j32 += 32) {
+                    const int64_t j = j32 + lane;
+                    const uint32_t word = fw[j32 >> 5];
+                    bool cap_now = false;
+                    if (j < w1 && !((word >> lane) & 1u)) {
+                        const float sv = vals[j];
+                        if (sv * near >= 1.f && lam * double(sv) >= 1.0) {
+                            cap_now = true;
+                            ++added_l;
+                            capped_l += double(sv);
+                        }
                     }
+                    const uint32_t nb = __ballot_sync(0xffffffffu, cap_now);
+                    if (nb != 0u && lane == 0) fw[j32 >> 5] = word | nb;
                 }
                 const int added = block_sum<int>(added_l, sc.iwarp, &sc.bcast[0]);
                 if (added == 0) break;
-                rest = block_sum<double>(rest_l, sc.dwarp, &sc.dbcast);
+                rest -= block_sum<double>(capped_l, sc.dwarp, &sc.dbcast);
                 ncap += added;
                 lam = (Bblk - double(ncap)) / rest;
             }
-            for (int64_t j = tid; j < nkvb; j += PL_THREADS)
-                vals[j] = (bits[j >> 5] >> (j & 31)) & 1u ? 1.f : __double2float_rn(lam * double(vals[j]));
+            // pi into shared memory (lane-strided, conflict-free); the capped
+            // flags are cleared again for the sampling pass
+            for (int64_t j32 = w0; j32 < w1; j32 += 32) {
+                const int64_t j = j32 + lane;
+                const uint32_t word = fw[j32 >> 5];
+                if (j < w1) vals[j] = ((word >> lane) & 1u) ? 1.f : __double2float_rn(lam * double(vals[j]));
+                __syncwarp();
+                if (lane == 0) fw[j32 >> 5] = 0u;
+            }
         }
-        __syncthreads();
-        if (pi_out != nullptr)
-            for (int64_t j = tid; j < nkvb; j += PL_THREADS) pi_out[row * nkvb + j] = vals[j];
-    } else {
-        __syncthreads();
     }
+    __syncthreads();
+    if (MODE == kPlanSip && pi_out != nullptr)
+        for (int64_t j = tid; j < nkvb; j += PL_THREADS) pi_out[row * nkvb + j] = vals[j];
 
     // top-k threshold: radix select on the fp32 bit patterns of the
     // non-negative scores, 8 bits per pass, most significant first
@@ -205,33 +242,28 @@ __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
         need_eq = kk;
     }
 
-    // ---- selection flags and per-warp counts (warp w owns a contiguous segment)
-    // Sampled modes keep their take flags as bits (the capping flags are done).
-    if (MODE != kPlanTopk) {
-        for (int w = tid; w < nwords; w += PL_THREADS) bits[w] = 0u;
-        __syncthreads();
-    }
-    const int64_t seg = ((nkvb + PL_WARPS * 128 - 1) / (PL_WARPS * 128)) * 128;
-    const int64_t w0 = int64_t(wid) * seg;
-    const int64_t w1 = w0 + seg < nkvb ? w0 + seg : nkvb;
+    // ---- pass 1: (SIP) final pi; flags <- taken blocks; per-warp counts
     int nsel_w = 0, neq_w = 0;
-    for (int64_t base = w0; base < w1; base += 128) {
-        const int64_t j0 = base + 4 * lane;
+    for (int64_t j0 = w0 + 8 * lane; j0 < w1; j0 += 256) {
         uint32_t tk = 0, ek = 0;
         if (MODE == kPlanTopk) {
+            float raw[8];
+            load8(vals, j0, w1, raw);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < 8; ++u) {
                 const int64_t j = j0 + u;
-                const uint32_t bv = j < w1 ? __float_as_uint(vals[j]) : 0u;
+                const uint32_t bv = __float_as_uint(raw[u]);
                 tk |= uint32_t(k_top > 0 && j < w1 && bv > thr) << u;
                 ek |= uint32_t(k_top > 0 && j < w1 && bv == thr) << u;
             }
-        } else if (j0 < w1) {
-            float u4[4];
-            row_uniforms(seed, b, h, qb, j0 >> 2, u4);
+        } else {
+            float pv[8];
+            load8(vals, j0, w1, pv);
+            float u8[8];
+            row_uniforms8(seed, b, h, qb, j0 >> 3, u8);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) tk |= uint32_t(j0 + u < w1 && u4[u] < vals[j0 + u]) << u;
-            if (tk) atomicOr(&bits[j0 >> 5], tk << (j0 & 31));
+            for (int u = 0; u < 8; ++u) tk |= uint32_t(j0 + u < w1 && u8[u] < pv[u]) << u;
+            flags[j0 >> 3] = uint8_t(tk);
         }
         nsel_w += __popc(tk);
         neq_w += __popc(ek);
@@ -254,21 +286,21 @@ __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
     }
     if (MODE == kPlanTopk) {
         // ties at the threshold are taken in ascending index order until k
-        const int64_t from_eq = eq_total < need_eq ? eq_total : need_eq;
-        pos += eq_rank < need_eq ? eq_rank : need_eq;  // ties of earlier warps taken before us
-        total += from_eq;
+        pos += eq_rank < need_eq ? eq_rank : need_eq;  // ties of earlier warps taken before ours
+        total += eq_total < need_eq ? eq_total : need_eq;
     }
 
-    // ---- compaction in ascending index order, warp by warp
-    for (int64_t base = w0; base < w1; base += 128) {
-        const int64_t j0 = base + 4 * lane;
+    // ---- pass 2: compaction in ascending index order within the warp's segment
+    for (int64_t j0 = w0 + 8 * lane; j0 < w1; j0 += 256) {
         uint32_t tk = 0;
         if (MODE == kPlanTopk) {
             uint32_t ek = 0;
+            float raw[8];
+            load8(vals, j0, w1, raw);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < 8; ++u) {
                 const int64_t j = j0 + u;
-                const uint32_t bv = j < w1 ? __float_as_uint(vals[j]) : 0u;
+                const uint32_t bv = __float_as_uint(raw[u]);
                 tk |= uint32_t(k_top > 0 && j < w1 && bv > thr) << u;
                 ek |= uint32_t(k_top > 0 && j < w1 && bv == thr) << u;
             }
@@ -281,15 +313,15 @@ __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
             }
             int64_t r = eq_rank + (incl - neq);  // rank of this lane's first tie
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < 8; ++u) {
                 if ((ek >> u) & 1u) {
                     if (r < need_eq) tk |= 1u << u;
                     ++r;
                 }
             }
             eq_rank += __shfl_sync(0xffffffffu, incl, 31);
-        } else if (j0 < w1) {
-            tk = (bits[j0 >> 5] >> (j0 & 31)) & 15u;
+        } else {
+            tk = flags[j0 >> 3];
         }
         const int nt = __popc(tk);
         int incl = nt;
@@ -300,7 +332,7 @@ __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
         }
         int64_t p = pos + (incl - nt);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < 8; ++u) {
             if ((tk >> u) & 1u) {
                 if (p < cap) {
                     idx_out[row * cap + p] = int32_t(j0 + u);

@@ -118,8 +118,9 @@ int abattn_score(const float *C, const float *w, const float *Kbar, const abattn
 /* Planner from scores ([P1] SIP bullet, [P2] SIP paragraph).
  * SIP: pi_j = min(1, lambda*s_j) with sum_j pi_j = budget*nKVB (capping
  * iteration, sums in fp64, pi rounded to fp32); block j is taken iff
- * u_j < pi_j in fp32, u_j the top 24 bits of word j%4 of
- * Philox4x64-10(counter (j/4, qb, h, b), key (seed, 0)) times 2^-24.
+ * u_j < pi_j in fp32, u_j = (top 24 bits of the high (even j) or low (odd
+ * j) 32-bit half of word (j/2)%4 of Philox4x64-10(counter (j/8, qb, h, b),
+ * key (seed, 0))) times 2^-24.
  * TOPK: the floor(budget*nKVB + 0.5) highest scores, ties to the lower
  * index, weight 1.
  * Outputs per row, indices ascending: counts int32 [rows], idx int32

@@ -195,16 +195,20 @@ void oc_philox4x64_10(const uint64_t ctr[4], const uint64_t key[2], uint64_t out
     out[0] = x0; out[1] = x1; out[2] = x2; out[3] = x3;
 }
 
-/* The uniform for KV block j of row (b, h, qb): counter (j / 4, qb, h, b),
- * key (seed, 0); word j % 4 supplies the draw, whose top 24 bits give
- * u = bits * 2^-24, exactly representable in float32 (READING).            */
+/* The uniform for KV block j of row (b, h, qb): counter (j / 8, qb, h, b),
+ * key (seed, 0); 64-bit word (j / 2) % 4 of the block supplies two draws, its
+ * high 32-bit half for even j and its low half for odd j; the top 24 bits of
+ * that half give u = bits * 2^-24, exactly representable in float32
+ * (READING: the pages name no generator).                                   */
 float oc_uniform(uint64_t seed, int64_t b, int64_t h, int64_t qb, int64_t j)
 {
-    uint64_t ctr[4] = {(uint64_t)(j >> 2), (uint64_t)qb, (uint64_t)h, (uint64_t)b};
+    uint64_t ctr[4] = {(uint64_t)(j >> 3), (uint64_t)qb, (uint64_t)h, (uint64_t)b};
     uint64_t key[2] = {seed, 0};
     uint64_t out[4];
     oc_philox4x64_10(ctr, key, out);
-    return (float)(out[j & 3] >> 40) * 0x1p-24f;
+    uint64_t w = out[(j >> 1) & 3];
+    uint32_t half = (j & 1) ? (uint32_t)w : (uint32_t)(w >> 32);
+    return (float)(half >> 8) * 0x1p-24f;
 }
 
 /* Poisson sampling.  [P2] SIP paragraph: each block enters the sample on its

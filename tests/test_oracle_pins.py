@@ -225,11 +225,13 @@ def test_philox_matches_numpy_bit_generator(key, ctr):
     np.testing.assert_array_equal(got, want)
 
 
-def test_uniform_uses_word_of_counter_block():
+def test_uniform_uses_halves_of_counter_block_words():
     seed, b, h, qb = 77, 0, 3, 5
-    for j in [0, 1, 2, 3, 4, 7, 1001]:
-        words = oracle.philox4x64_10([j // 4, qb, h, b], [seed, 0])
-        assert oracle.uniform(seed, b, h, qb, j) == float(int(words[j % 4]) >> 40) * 2.0**-24
+    for j in [0, 1, 2, 3, 4, 7, 8, 9, 1001]:
+        words = oracle.philox4x64_10([j // 8, qb, h, b], [seed, 0])
+        w = int(words[(j // 2) % 4])
+        half = (w & 0xFFFFFFFF) if j % 2 else (w >> 32)
+        assert oracle.uniform(seed, b, h, qb, j) == float(half >> 8) * 2.0**-24
 
 
 def test_uniform_statistics():
