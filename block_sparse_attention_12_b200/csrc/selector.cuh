@@ -275,10 +275,15 @@ __global__ void __launch_bounds__(KM_THREADS) kmeans_kernel(
 //   pass 2, operands swapped, rows = KV blocks: each thread owns one KV block
 //           j and writes s_j = sum_c (w_c / Z_c) 2^(L_cj - m_c) for the 16
 //           q-blocks (the 8 clusters of a q-block are 8 columns of its row).
-// Warp 0 streams the Kbar tiles by TMA (2 stages), warp 1 issues the MMAs
-// into two TMEM accumulators, warps 2..5 run the epilogue.  Logits are in
-// log2 units.
-constexpr int SC_THREADS = 192;
+// Warps 0..7 are two epilogue warpgroups taking alternate tiles (TMEM
+// accumulator u % 2); at the end of pass 1 they merge their per-centroid
+// (max, normaliser).  Warp 8 streams the Kbar tiles by TMA (2 stages), warp 9
+// issues the MMAs.  Logits are in log2 units.
+constexpr int SC_THREADS = 384;
+constexpr int SC_EPI_REGS = 216;    // setmaxnreg of the two epilogue warpgroups
+constexpr int SC_OTHER_REGS = 64;   // producer / MMA warpgroup
+static_assert(2 * 128 * SC_EPI_REGS + 128 * SC_OTHER_REGS <= SC_THREADS * 168,
+              "setmaxnreg split exceeds the launch register budget");
 constexpr int SC_QBT = 16;  // q-blocks per CTA (x 8 cluster slots = 128 rows)
 
 template <int D>
@@ -288,8 +293,9 @@ struct ScoreLayout {
     static constexpr int C_HI = 0;
     static constexpr int C_LO = TILE;
     static constexpr int STAGE0 = 2 * TILE;  // stage s: hi at STAGE0 + 2*s*TILE, lo right after
-    static constexpr int MC_OFF = STAGE0 + 4 * TILE;
-    static constexpr int BAR_OFF = MC_OFF + 2 * 128 * 4;
+    static constexpr int MC_OFF = STAGE0 + 4 * TILE;       // m[128], coef[128]
+    static constexpr int XCH_OFF = MC_OFF + 2 * 128 * 4;   // odd warpgroup's pass-1 (m, z)[128]
+    static constexpr int BAR_OFF = XCH_OFF + 2 * 128 * 4;
     static constexpr int NBARS = 9;
     static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
     static constexpr int BYTES = MISC_OFF + 16;
@@ -305,7 +311,8 @@ struct ScoreParams {
     float scale_log2;
 };
 
-__device__ __forceinline__ void epi_bar_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void epi_bar_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
 
 template <int D>
 __global__ void __launch_bounds__(SC_THREADS, 1)
@@ -321,11 +328,12 @@ __global__ void __launch_bounds__(SC_THREADS, 1)
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::BAR_OFF);
     uint64_t *c_full = bars, *kv_full = bars + 1, *kv_empty = bars + 3, *acc_full = bars + 5,
              *acc_free = bars + 7;
+    float *xch = reinterpret_cast<float *>(smem + L::XCH_OFF);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::MISC_OFF);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::MISC_OFF + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int g = blockIdx.x, bh = blockIdx.y;
+    const int ct = blockIdx.x, bh = blockIdx.y;  // centroid tile (16 q-blocks), head
     const int NT = (p.nkvb + 127) / 128;
     const int U = 2 * NT;  // tile visits over both passes
 
@@ -340,7 +348,7 @@ __global__ void __launch_bounds__(SC_THREADS, 1)
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 1) {
+    if (warp == 9) {
         tmem_alloc(tmem_slot, 256);
         tmem_relinquish();
     }
@@ -349,13 +357,14 @@ __global__ void __launch_bounds__(SC_THREADS, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 0) {
+    if (warp == 8) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(SC_OTHER_REGS) : "memory");
         if (lane == 0) {
             mbar_arrive_expect_tx(c_full, 2 * L::TILE);
 #pragma unroll
             for (int h = 0; h < L::HALVES; ++h) {
-                tma_load_3d(smem + L::C_HI + h * 16384, &tmChi, c_full, h * 64, g * 128, bh);
-                tma_load_3d(smem + L::C_LO + h * 16384, &tmClo, c_full, h * 64, g * 128, bh);
+                tma_load_3d(smem + L::C_HI + h * 16384, &tmChi, c_full, h * 64, ct * 128, bh);
+                tma_load_3d(smem + L::C_LO + h * 16384, &tmClo, c_full, h * 64, ct * 128, bh);
             }
             int issued = 0;
             for (int u = 0; u < U; ++u) {
@@ -376,8 +385,9 @@ __global__ void __launch_bounds__(SC_THREADS, 1)
             }
         }
         __syncwarp();
-    } else if (warp == 1) {
-        if (lane == 0) {
+    } else if (warp >= 9) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(SC_OTHER_REGS) : "memory");
+        if (warp == 9 && lane == 0) {
             constexpr uint32_t idesc = make_idesc_bf16(128, 128, 0, 0);
             const uint32_t cb = smem_u32(smem);
             bool ok = mbar_wait(c_full, 0, abort_flag);
@@ -405,85 +415,109 @@ __global__ void __launch_bounds__(SC_THREADS, 1)
         }
         __syncwarp();
     } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(SC_EPI_REGS) : "memory");
+        const int eg = warp >> 2;  // this warpgroup takes tiles u with u % 2 == eg
         const int wq = warp & 3, rr = wq * 32 + lane;
-        const uint32_t t_lane = tmem + (uint32_t(wq * 32) << 16);
-        float m = -INFINITY, z = 0.f;
+        const uint32_t t_lane = tmem + (uint32_t(wq * 32) << 16) + eg * 128;
+        float m = -INFINITY, z = 0.f;  // pass 1: raw-accumulator max and sum of 2^(s*(L - m))
         bool ok = true;
-        for (int u = 0; u < U; ++u) {
-            const int b = u & 1;
-            if (u == NT) {
-                // pass-1 statistics of this thread's centroid row -> shared memory
-                const int qb = g * SC_QBT + (rr >> 3), c = rr & 7;
-                float coef = 0.f;
-                if (qb < p.nqb && c < p.nc) {
-                    const float wc = p.w[(int64_t(bh) * p.nqb + qb) * p.nc + c];
-                    if (wc > 0.f && z > 0.f) coef = wc / z;
-                }
-                sm_m[rr] = m;
-                sm_coef[rr] = coef;
-                epi_bar_sync();
-            }
-            // on an abort every thread still runs all iterations (without
-            // work) so that all of them reach the named barrier above
-            if (!ok || !mbar_wait(&acc_full[b], (u >> 1) & 1, abort_flag)) { ok = false; continue; }
+        const float sl2 = p.scale_log2;
+        // reads this warpgroup's accumulator of tile u into x; false on abort
+        auto fetch_acc = [&](int u, uint32_t (&x)[4][32]) -> bool {
+            if (!ok || !mbar_wait(&acc_full[eg], (u >> 1) & 1, abort_flag)) { ok = false; return false; }
             tc_fence_after();
-            uint32_t x[4][32];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(t_lane + b * 128 + c * 32, x[c]);
+            for (int c = 0; c < 4; ++c) tmem_ld32(t_lane + c * 32, x[c]);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_free[b]);
-            if (u < NT) {
-                // pass 1: columns are KV blocks u*128 + col
-                const int j0 = u * 128;
-                float mt = -INFINITY;
+            if (lane == 0) mbar_arrive(&acc_free[eg]);
+            return true;
+        };
+        // ---- pass 1: columns are KV blocks u*128 + col
+        for (int u = eg; u < NT; u += 2) {
+            uint32_t x[4][32];
+            if (!fetch_acc(u, x)) continue;
+            const int j0 = u * 128;
+            if (j0 + 128 > p.nkvb) {
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const float v = j0 + c * 32 + i < p.nkvb ? __uint_as_float(x[c][i]) * p.scale_log2 : -INFINITY;
-                        x[c][i] = __float_as_uint(v);
-                        mt = fmaxf(mt, v);
-                    }
-                const float mn = fmaxf(m, mt);
-                if (mn != -INFINITY) {
-                    float acc = 0.f;
+                    for (int i = 0; i < 32; ++i)
+                        if (j0 + c * 32 + i >= p.nkvb) x[c][i] = __float_as_uint(-INFINITY);
+            }
+            float mt0 = -INFINITY, mt1 = -INFINITY;
 #pragma unroll
-                    for (int c = 0; c < 4; ++c)
+            for (int c = 0; c < 4; ++c)
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) acc += exp2f(__uint_as_float(x[c][i]) - mn);
-                    z = z * exp2f(m - mn) + acc;
-                    m = mn;
+                for (int i = 0; i < 32; i += 2) {
+                    mt0 = fmaxf(mt0, __uint_as_float(x[c][i]));
+                    mt1 = fmaxf(mt1, __uint_as_float(x[c][i + 1]));
                 }
-            } else {
-                // pass 2: this thread's row is KV block j; columns are centroid rows
-                const int j = (u - NT) * 128 + rr;
+            const float mn = fmaxf(m, fmaxf(mt0, mt1));
+            if (mn != -INFINITY) {
+                const float neg = -mn * sl2;
+                float a[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int q = 0; q < SC_QBT; ++q) {
-                    const float4 m0 = *reinterpret_cast<const float4 *>(sm_m + q * 8);
-                    const float4 m1 = *reinterpret_cast<const float4 *>(sm_m + q * 8 + 4);
-                    const float4 k0 = *reinterpret_cast<const float4 *>(sm_coef + q * 8);
-                    const float4 k1 = *reinterpret_cast<const float4 *>(sm_coef + q * 8 + 4);
-                    const float mm[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
-                    const float kk[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
-                    float sv = 0.f;
+                for (int c = 0; c < 4; ++c)
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const float lv = __uint_as_float(x[q >> 2][(q & 3) * 8 + c]) * p.scale_log2;
-                        if (kk[c] != 0.f) sv = fmaf(kk[c], exp2f(lv - mm[c]), sv);
-                    }
-                    const int qb = g * SC_QBT + q;
-                    if (j < p.nkvb && qb < p.nqb) p.S[(int64_t(bh) * p.nqb + qb) * p.nkvb + j] = sv;
-                }
+                    for (int i = 0; i < 32; ++i) a[i & 3] += fast_exp2(fmaf(__uint_as_float(x[c][i]), sl2, neg));
+                z = (m == -INFINITY ? 0.f : z * fast_exp2((m - mn) * sl2)) + ((a[0] + a[1]) + (a[2] + a[3]));
+                m = mn;
             }
         }
-        (void)ok;
+        // ---- merge of the two warpgroups' statistics (every epilogue thread
+        // reaches both barriers, whatever its number of tiles)
+        if (eg == 1) {
+            xch[rr] = m;
+            xch[128 + rr] = z;
+        }
+        epi_bar_sync();
+        if (eg == 0) {
+            const float m1 = xch[rr], z1 = xch[128 + rr];
+            const float mm = fmaxf(m, m1);
+            float zz = 0.f;
+            if (mm != -INFINITY) {
+                if (m != -INFINITY) zz += z * fast_exp2((m - mm) * sl2);
+                if (m1 != -INFINITY) zz += z1 * fast_exp2((m1 - mm) * sl2);
+            }
+            const int qb = ct * SC_QBT + (rr >> 3), c = rr & 7;
+            float coef = 0.f, mlog = 0.f;  // a padding slot: weight 0 against 2^(s*L)
+            if (qb < p.nqb && c < p.nc && zz > 0.f) {
+                const float wc = p.w[(int64_t(bh) * p.nqb + qb) * p.nc + c];
+                coef = wc / zz;
+                mlog = mm * sl2;
+            }
+            sm_m[rr] = mlog;
+            sm_coef[rr] = coef;
+        }
+        epi_bar_sync();
+        // ---- pass 2: this thread's row is KV block j; columns are centroid rows
+        for (int u = NT + ((eg - NT) & 1); u < U; u += 2) {
+            uint32_t x[4][32];
+            if (!fetch_acc(u, x)) continue;
+            const int j = (u - NT) * 128 + rr;
+#pragma unroll
+            for (int q = 0; q < SC_QBT; ++q) {
+                const float4 m0 = *reinterpret_cast<const float4 *>(sm_m + q * 8);
+                const float4 m1 = *reinterpret_cast<const float4 *>(sm_m + q * 8 + 4);
+                const float4 k0 = *reinterpret_cast<const float4 *>(sm_coef + q * 8);
+                const float4 k1 = *reinterpret_cast<const float4 *>(sm_coef + q * 8 + 4);
+                const float mm[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+                const float kk[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+                float sv = 0.f;
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    sv = fmaf(kk[c], fast_exp2(fmaf(__uint_as_float(x[q >> 2][(q & 3) * 8 + c]), sl2, -mm[c])), sv);
+                const int qb = ct * SC_QBT + q;
+                if (j < p.nkvb && qb < p.nqb) p.S[(int64_t(bh) * p.nqb + qb) * p.nkvb + j] = sv;
+            }
+        }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == 9) {
         tc_fence_after();
         tmem_dealloc(tmem, 256);
     }
