@@ -35,7 +35,7 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-from block_sparse_attention_12_b200 import inputs  # noqa: E402
+from block_sparse_attention_12_b200 import inputs, multigpu  # noqa: E402
 
 METRIC = "AB-Attn fwd ms & executed TFLOPS (% bf16 TC peak), 75.6K tok × 40 heads"
 UNIT = "TFLOP/s"
@@ -45,7 +45,7 @@ FP32_LANES_PER_SM = 128
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="wan14b-720p", choices=sorted(inputs.WORKLOADS))
@@ -357,13 +357,9 @@ def main():
     if dist:
         dist.barrier()
     clk = clocks.stop()
-    ms = e0.elapsed_time(e1) / args.steps
-    if dist:
-        t = torch.tensor([ms], device=Q.device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = multigpu.max_over_ranks(e0.elapsed_time(e1) / args.steps, Q.device)
     abi.check()
-    value = exec_fl * world / (ms / 1e3) / 1e12
+    value = multigpu.job_throughput(exec_fl, ms, world) / 1e12
 
     # ---- per-kernel breakdown (separate loops, same stream, after the timed region)
     kb_ms = {}
@@ -449,13 +445,9 @@ def main():
         torch.cuda.synchronize()
         if dist:
             dist.barrier()
-        e2e_ms = timed(e2e_step, args.e2e_steps, stream)
-        if dist:
-            t = torch.tensor([e2e_ms], device=Q.device)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = multigpu.max_over_ranks(timed(e2e_step, args.e2e_steps, stream), Q.device)
         abi.check()
-        e2e = {"value": exec_fl * world / (e2e_ms / 1e3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
+        e2e = {"value": multigpu.job_throughput(exec_fl, e2e_ms, world) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": 3 * Q.numel() * Q.element_size(),
                "d2h_bytes_per_step": O.numel() * O.element_size()}
         del Qh, Kh, Vh, Oh, Qd, Kd, Vd

@@ -224,7 +224,7 @@ int launch_plan(int mode, const float *in, const abattn_dims *d, const abattn_pa
     const double Bblk = double(p->budget) * double(nkvb);
     int64_t k_top = int64_t(floor(Bblk + 0.5));
     if (k_top > nkvb) k_top = nkvb;
-    const size_t smem = sizeof(float) * nkvb + 4 * size_t((nkvb + 31) / 32);
+    const size_t smem = sizeof(float) * nkvb + 4 * size_t((nkvb + 31) / 32);  // scores, flag words
     cudaError_t e;
     switch (mode) {
         case kPlanSip:

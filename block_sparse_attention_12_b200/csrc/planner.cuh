@@ -84,6 +84,28 @@ struct PlanScratch {
     int hist[256];
 };
 
+// Block-wide sums of one int and one double in a single exchange.
+__device__ __forceinline__ void block_sum2(int vi, double vd, PlanScratch &sc, int &si, double &sd) {
+    vi = warp_sum(vi);
+    vd = warp_sum(vd);
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    if (lane == 0) {
+        sc.iwarp[wid] = vi;
+        sc.dwarp[wid] = vd;
+    }
+    __syncthreads();
+    int ti = 0;
+    double td = 0.0;
+#pragma unroll
+    for (int w = 0; w < PL_WARPS; ++w) {
+        ti += sc.iwarp[w];
+        td += sc.dwarp[w];
+    }
+    si = ti;
+    sd = td;
+    __syncthreads();
+}
+
 // Block-wide sum; every thread gets the result.
 template <typename T>
 __device__ __forceinline__ T block_sum(T v, T *warp_buf, T *bcast) {
@@ -172,24 +194,35 @@ __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
                 const float near = float(lam) * (1.f + 1e-5f);
                 int added_l = 0;
                 double capped_l = 0.0;
-                for (int64_t j32 = w0; j32 < w1; j32 += 32) {
-                    const int64_t j = j32 + lane;
-                    const uint32_t word = fw[j32 >> 5];
-                    bool cap_now = false;
-                    if (j < w1 && !((word >> lane) & 1u)) {
-                        const float sv = vals[j];
-                        if (sv * near >= 1.f && lam * double(sv) >= 1.0) {
+                // four words (128 blocks) per step: four independent chains
+                for (int64_t j128 = w0; j128 < w1; j128 += 128) {
+                    uint32_t word[4];
+                    float sv[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int64_t j = j128 + 32 * q + lane;
+                        word[q] = j128 + 32 * q < w1 ? fw[(j128 >> 5) + q] : 0xFFFFFFFFu;
+                        sv[q] = j < w1 ? vals[j] : 0.f;
+                    }
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int64_t j = j128 + 32 * q + lane;
+                        bool cap_now = false;
+                        if (j < w1 && !((word[q] >> lane) & 1u) && sv[q] * near >= 1.f &&
+                            lam * double(sv[q]) >= 1.0) {
                             cap_now = true;
                             ++added_l;
-                            capped_l += double(sv);
+                            capped_l += double(sv[q]);
                         }
+                        const uint32_t nb = __ballot_sync(0xffffffffu, cap_now);
+                        if (nb != 0u && lane == 0) fw[(j128 >> 5) + q] = word[q] | nb;
                     }
-                    const uint32_t nb = __ballot_sync(0xffffffffu, cap_now);
-                    if (nb != 0u && lane == 0) fw[j32 >> 5] = word | nb;
                 }
-                const int added = block_sum<int>(added_l, sc.iwarp, &sc.bcast[0]);
+                int added;
+                double capped;
+                block_sum2(added_l, capped_l, sc, added, capped);
                 if (added == 0) break;
-                rest -= block_sum<double>(capped_l, sc.dwarp, &sc.dbcast);
+                rest -= capped;
                 ncap += added;
                 lam = (Bblk - double(ncap)) / rest;
             }

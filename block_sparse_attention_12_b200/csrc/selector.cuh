@@ -203,8 +203,12 @@ __global__ void __launch_bounds__(KM_THREADS) kmeans_kernel(
                 const float v = fmaf(-2.f, a[c], cn[c]);
                 if (c < nc && v < bd) { bd = v; best = c; }
             }
-            lab[tid] = best;
         }
+        // a fixed point (no label changed) repeats itself in every remaining
+        // iteration: stop, the result is the same as running them all
+        const bool moved = tid < M && (it == 0 || lab[tid] != best);
+        if (it > 0 && !__syncthreads_or(moved)) break;
+        if (tid < M) lab[tid] = best;
         // stable counting sort of the labels
         unsigned my_rank = 0;
 #pragma unroll
