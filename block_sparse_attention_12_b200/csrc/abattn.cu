@@ -246,18 +246,29 @@ int launch_plan(int mode, const float *in, const abattn_dims *d, const abattn_pa
     return launch_status();
 }
 
-template <int HD, bool DENSE>
+template <int HD, bool DENSE, bool GROUPED>
 int launch_fwd_t(const CUtensorMap &mQ, const CUtensorMap &mK, const CUtensorMap &mV, const FwdParams &fp,
                  int64_t rows, cudaStream_t st) {
     constexpr int smem = FwdLayout<HD>::ALLOC;
     static bool attr = false;
     if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(fwd_kernel<HD, DENSE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        cudaError_t e =
+            cudaFuncSetAttribute(fwd_kernel<HD, DENSE, GROUPED>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return cuda_status(e);
         attr = true;
     }
-    fwd_kernel<HD, DENSE><<<unsigned(rows), FWD_THREADS, smem, st>>>(mQ, mK, mV, fp);
+    fwd_kernel<HD, DENSE, GROUPED><<<unsigned(rows), FWD_THREADS, smem, st>>>(mQ, mK, mV, fp);
     return launch_status();
+}
+
+template <int HD>
+int launch_fwd_hd(bool dense, bool grouped, const CUtensorMap &mQ, const CUtensorMap &mK, const CUtensorMap &mV,
+                  const FwdParams &fp, int64_t rows, cudaStream_t st) {
+    if (dense)
+        return grouped ? launch_fwd_t<HD, true, true>(mQ, mK, mV, fp, rows, st)
+                       : launch_fwd_t<HD, true, false>(mQ, mK, mV, fp, rows, st);
+    return grouped ? launch_fwd_t<HD, false, true>(mQ, mK, mV, fp, rows, st)
+                   : launch_fwd_t<HD, false, false>(mQ, mK, mV, fp, rows, st);
 }
 
 int run_forward(bool dense, const void *Q, const void *K, const void *V, const abattn_dims *d, int kb,
@@ -283,9 +294,11 @@ int run_forward(bool dense, const void *Q, const void *K, const void *V, const a
     fp.nkvb = int(cdiv(d->N, fp.kb));
     fp.scale_log2 = resolve_scale(scale, d->d) * 1.4426950408889634f;
     const int64_t rows = d->B * d->H * fp.nqb;
-    if (d->d == 128)
-        return dense ? launch_fwd_t<128, true>(mQ, mK, mV, fp, rows, st) : launch_fwd_t<128, false>(mQ, mK, mV, fp, rows, st);
-    return dense ? launch_fwd_t<64, true>(mQ, mK, mV, fp, rows, st) : launch_fwd_t<64, false>(mQ, mK, mV, fp, rows, st);
+    // every kv block starts at a multiple of 4 keys (kb is 4, 8, ..., 128), so
+    // with N % 4 == 0 each 4-key group of a tile is entirely valid or entirely past N
+    const bool grouped = (d->N % 4) == 0;
+    if (d->d == 128) return launch_fwd_hd<128>(dense, grouped, mQ, mK, mV, fp, rows, st);
+    return launch_fwd_hd<64>(dense, grouped, mQ, mK, mV, fp, rows, st);
 }
 
 int check_plan_shape(const abattn_dims *d, const abattn_params *p) {

@@ -84,7 +84,8 @@ struct FwdLayout {
     static constexpr int K_OFF = Q_OFF + TILE;
     static constexpr int V_OFF = K_OFF + FWD_NS * TILE;
     static constexpr int BIAS_OFF = V_OFF + FWD_NS * TILE;
-    static constexpr int BAR_OFF = BIAS_OFF + FWD_NS * 128 * 4;
+    static constexpr int GBIAS_OFF = BIAS_OFF + FWD_NS * 128 * 4;  // per 4-key group: [NS][32]
+    static constexpr int BAR_OFF = GBIAS_OFF + FWD_NS * 32 * 4;
     static constexpr int NBARS = 1 + 2 * FWD_NS + 6;
     // (m, l) of both softmax warpgroups, [2][2][128] floats, exchanged in the
     // epilogue through the first K stage: by then every QK^T MMA has completed
@@ -95,7 +96,10 @@ struct FwdLayout {
     static constexpr int ALLOC = BYTES + 1024;  // slack for 1024-byte alignment
 };
 
-template <int HD, bool DENSE>
+// GROUPED (N % 4 == 0): every 4-key group of a tile shares one bias, since
+// block boundaries are multiples of 4 keys and so is N; the softmax then adds
+// the bias once per group.  Otherwise the bias is kept per key.
+template <int HD, bool DENSE, bool GROUPED>
 __global__ void __launch_bounds__(FWD_THREADS, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -107,6 +111,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
     uint8_t *sK = smem + L::K_OFF;
     uint8_t *sV = smem + L::V_OFF;
     float *sBias = reinterpret_cast<float *>(smem + L::BIAS_OFF);
+    float *sGBias = reinterpret_cast<float *>(smem + L::GBIAS_OFF);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::BAR_OFF);
     uint64_t *q_full = bars;
     uint64_t *kv_full = bars + 1;
@@ -226,14 +231,21 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                         blk = fill_blk;  // padding slot: loaded, weighted zero
                     }
                     const int key0 = blk * kb + ro;
-                    float *bdst = sBias + s * 128 + unit * R;
-                    for (int i = 0; i < R; i += 4) {
-                        float4 v;
-                        v.x = key0 + i + 0 < p.N ? b : -INFINITY;
-                        v.y = key0 + i + 1 < p.N ? b : -INFINITY;
-                        v.z = key0 + i + 2 < p.N ? b : -INFINITY;
-                        v.w = key0 + i + 3 < p.N ? b : -INFINITY;
-                        *reinterpret_cast<float4 *>(bdst + i) = v;
+                    if constexpr (GROUPED) {
+                        // scalar stores: a unit's groups start at a multiple of R / 4
+                        // floats, which is 16-byte aligned only for R >= 16
+                        float *gdst = sGBias + s * 32 + unit * (R / 4);
+                        for (int i = 0; i < R; i += 4) gdst[i / 4] = key0 + i < p.N ? b : -INFINITY;
+                    } else {
+                        float *bdst = sBias + s * 128 + unit * R;
+                        for (int i = 0; i < R; i += 4) {
+                            float4 v;
+                            v.x = key0 + i + 0 < p.N ? b : -INFINITY;
+                            v.y = key0 + i + 1 < p.N ? b : -INFINITY;
+                            v.z = key0 + i + 2 < p.N ? b : -INFINITY;
+                            v.w = key0 + i + 3 < p.N ? b : -INFINITY;
+                            *reinterpret_cast<float4 *>(bdst + i) = v;
+                        }
                     }
                     __syncwarp(__activemask());
                     if (lane == 0) mbar_arrive_expect_tx(&kv_full[s], tx_bytes);
@@ -329,23 +341,43 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
             for (int c = 0; c < 4; ++c) tmem_ld32(t_S + c * 32, x[c]);
             tmem_wait_ld();
 
-            const float *bias = sBias + s * 128;
             float mt0 = -INFINITY, mt1 = -INFINITY;
+            const float *gbias = sGBias + s * 32;
+            if constexpr (GROUPED) {
+                // one bias per group of 4 keys (scale > 0): the row max is taken on
+                // the raw group maxima, one FFMA per group
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+                for (int q0 = 0; q0 < 32; q0 += 4) {
+                    const float4 g4 = *reinterpret_cast<const float4 *>(gbias + q0);
+                    const float gbq[4] = {g4.x, g4.y, g4.z, g4.w};
 #pragma unroll
-                for (int i = 0; i < 32; i += 4) {
-                    const float4 bb = *reinterpret_cast<const float4 *>(bias + c * 32 + i);
-                    const float v0 = fmaf(__uint_as_float(x[c][i + 0]), p.scale_log2, bb.x);
-                    const float v1 = fmaf(__uint_as_float(x[c][i + 1]), p.scale_log2, bb.y);
-                    const float v2 = fmaf(__uint_as_float(x[c][i + 2]), p.scale_log2, bb.z);
-                    const float v3 = fmaf(__uint_as_float(x[c][i + 3]), p.scale_log2, bb.w);
-                    x[c][i + 0] = __float_as_uint(v0);
-                    x[c][i + 1] = __float_as_uint(v1);
-                    x[c][i + 2] = __float_as_uint(v2);
-                    x[c][i + 3] = __float_as_uint(v3);
-                    mt0 = fmaxf(mt0, fmaxf(v0, v1));
-                    mt1 = fmaxf(mt1, fmaxf(v2, v3));
+                    for (int j = 0; j < 4; ++j) {
+                        const int q = q0 + j, c = q >> 3, i = (q & 7) * 4;
+                        const float gm = fmaxf(fmaxf(__uint_as_float(x[c][i]), __uint_as_float(x[c][i + 1])),
+                                               fmaxf(__uint_as_float(x[c][i + 2]), __uint_as_float(x[c][i + 3])));
+                        const float v = fmaf(gm, p.scale_log2, gbq[j]);
+                        if (j & 1) mt1 = fmaxf(mt1, v);
+                        else mt0 = fmaxf(mt0, v);
+                    }
+                }
+            } else {
+                const float *bias = sBias + s * 128;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4) {
+                        const float4 bb = *reinterpret_cast<const float4 *>(bias + c * 32 + i);
+                        const float v0 = fmaf(__uint_as_float(x[c][i + 0]), p.scale_log2, bb.x);
+                        const float v1 = fmaf(__uint_as_float(x[c][i + 1]), p.scale_log2, bb.y);
+                        const float v2 = fmaf(__uint_as_float(x[c][i + 2]), p.scale_log2, bb.z);
+                        const float v3 = fmaf(__uint_as_float(x[c][i + 3]), p.scale_log2, bb.w);
+                        x[c][i + 0] = __float_as_uint(v0);
+                        x[c][i + 1] = __float_as_uint(v1);
+                        x[c][i + 2] = __float_as_uint(v2);
+                        x[c][i + 3] = __float_as_uint(v3);
+                        mt0 = fmaxf(mt0, fmaxf(v0, v1));
+                        mt1 = fmaxf(mt1, fmaxf(v2, v3));
+                    }
                 }
             }
             const float m_new = fmaxf(m, fmaxf(mt0, mt1));
@@ -359,13 +391,32 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
             const bool any = __any_sync(0xffffffffu, need);
             const float m_use = (m == -INFINITY) ? 0.f : m;
             float rs[4] = {0.f, 0.f, 0.f, 0.f};
+            if constexpr (GROUPED) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+                for (int q0 = 0; q0 < 32; q0 += 4) {
+                    const float4 g4 = *reinterpret_cast<const float4 *>(gbias + q0);
+                    const float gbq[4] = {g4.x, g4.y, g4.z, g4.w};
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float e = fast_exp2(__uint_as_float(x[c][i]) - m_use);
-                    rs[i & 3] += e;
-                    x[c][i] = __float_as_uint(e);
+                    for (int j = 0; j < 4; ++j) {
+                        const int q = q0 + j, c = q >> 3, i = (q & 7) * 4;
+                        const float off = gbq[j] - m_use;
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const float e = fast_exp2(fmaf(__uint_as_float(x[c][i + k]), p.scale_log2, off));
+                            rs[k] += e;
+                            x[c][i + k] = __float_as_uint(e);
+                        }
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const float e = fast_exp2(__uint_as_float(x[c][i]) - m_use);
+                        rs[i & 3] += e;
+                        x[c][i] = __float_as_uint(e);
+                    }
                 }
             }
             l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
@@ -380,12 +431,14 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                 }
                 tmem_st32(t_S + c * 16, pk);
             }
-            if (ntiles > 0) {
-                // this warpgroup's O must be complete before it is rescaled;
-                // PV(t) is issued only after p_full below
+            if (ntiles > 0 && any) {
+                // this warpgroup's O must be complete before it is rescaled
+                // (PV(t) is issued only after p_full below).  Waiting only when
+                // rescaling is safe: PV(t) needs our p_full(t), so the barrier is
+                // never more than one phase past the one waited for.
                 if (!mbar_wait(&pv_done[g], ((t >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-                if (any) {
+                {
 #pragma unroll
                     for (int c = 0; c < HD / 32; ++c) {
                         uint32_t o[32];
