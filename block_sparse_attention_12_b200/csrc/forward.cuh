@@ -47,10 +47,10 @@ constexpr int FWD_THREADS = 512;
 // the producer and MMA warpgroups FWD_OTHER_REGS; 2*128*S + 2*128*O must not
 // exceed the 512 x 128 registers the CTA launches with.
 #ifndef ABATTN_FWD_SOFTMAX_REGS
-#define ABATTN_FWD_SOFTMAX_REGS 208
+#define ABATTN_FWD_SOFTMAX_REGS 200
 #endif
 #ifndef ABATTN_FWD_OTHER_REGS
-#define ABATTN_FWD_OTHER_REGS 48
+#define ABATTN_FWD_OTHER_REGS 56
 #endif
 constexpr int FWD_SOFTMAX_REGS = ABATTN_FWD_SOFTMAX_REGS;
 constexpr int FWD_OTHER_REGS = ABATTN_FWD_OTHER_REGS;
@@ -83,9 +83,11 @@ struct FwdLayout {
     static constexpr int Q_OFF = 0;
     static constexpr int K_OFF = Q_OFF + TILE;
     static constexpr int V_OFF = K_OFF + FWD_NS * TILE;
+    // per-key bias [NS][128] (N % 4 != 0) or per-group bias [NS][32]: one
+    // kernel uses one of the two, so they share the area
     static constexpr int BIAS_OFF = V_OFF + FWD_NS * TILE;
-    static constexpr int GBIAS_OFF = BIAS_OFF + FWD_NS * 128 * 4;  // per 4-key group: [NS][32]
-    static constexpr int BAR_OFF = GBIAS_OFF + FWD_NS * 32 * 4;
+    static constexpr int GBIAS_OFF = BIAS_OFF;
+    static constexpr int BAR_OFF = BIAS_OFF + FWD_NS * 128 * 4;
     static constexpr int NBARS = 1 + 2 * FWD_NS + 6;
     // (m, l) of both softmax warpgroups, [2][2][128] floats, exchanged in the
     // epilogue through the first K stage: by then every QK^T MMA has completed
@@ -204,13 +206,27 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                     pi = __ldg(rpi + e);
                 }
             };
+            if (!DENSE) {
+                // the plan row is read once per tile by every producer lane:
+                // bring it into L1 up front
+                const int lines = (cnt * 4 + 127) / 128;
+                for (int i = pw * 32 + lane; i < 2 * lines; i += FWD_PRODUCERS * 32)
+                    prefetch_l1(i < lines ? reinterpret_cast<const char *>(ridx) + i * 128
+                                          : reinterpret_cast<const char *>(rpi) + (i - lines) * 128);
+            }
+            // plan entries of tiles t (cur) and t+1 (nxt); the entry of tile
+            // t+2 is fetched at the top of iteration t
             int cur_blk, nxt_blk;
             float cur_pi, nxt_pi;
             fetch(0, cur_blk, cur_pi);
+            fetch(1, nxt_blk, nxt_pi);
             for (int t = 0; t < T; ++t) {
                 const int s = t % FWD_NS;
-                fetch(t + 1, nxt_blk, nxt_pi);
+                int x_blk;
+                float x_pi;
+                fetch(t + 2, x_blk, x_pi);
                 if (t >= FWD_NS && !mbar_wait(&kv_empty[s], ((t / FWD_NS) - 1) & 1, abort_flag)) break;
+                int key0 = 0;
                 if (owner) {
                     // block of this unit, its validity and the bias of its R keys
                     int blk;
@@ -230,7 +246,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                     } else {
                         blk = fill_blk;  // padding slot: loaded, weighted zero
                     }
-                    const int key0 = blk * kb + ro;
+                    key0 = blk * kb + ro;
                     if constexpr (GROUPED) {
                         // scalar stores: a unit's groups start at a multiple of R / 4
                         // floats, which is 16-byte aligned only for R >= 16
@@ -263,6 +279,8 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                 __syncwarp();
                 cur_blk = nxt_blk;
                 cur_pi = nxt_pi;
+                nxt_blk = x_blk;
+                nxt_pi = x_pi;
                 ++issued;
             }
             // drain: every issued copy lands before the CTA may exit
@@ -282,16 +300,18 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
             constexpr uint32_t idesc_pv = make_idesc_bf16(128, HD, 0, 1);
             const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
             bool ok = mbar_wait(q_full, 0, abort_flag);
+            // descriptor low words (see umma_ss_lo): K-major operands have LBO 16,
+            // V as an MN-major operand LBO 16384 (its second 64-column half)
+            const uint32_t q_lo = sdesc_lo(aQ, 16), k_lo = sdesc_lo(aK, 16), v_lo = sdesc_lo(aV, 16384);
             auto issue_qk = [&](int t) -> bool {
                 const int s = t % FWD_NS, sb = t & 1;
                 if (!mbar_wait(&kv_full[s], (t / FWD_NS) & 1, abort_flag)) return false;
                 tc_fence_after();
-                const uint32_t kbase = aK + s * L::TILE;
+                const uint32_t kb_lo = k_lo + uint32_t(s) * (L::TILE >> 4);
 #pragma unroll
                 for (int k = 0; k < HD / 16; ++k) {
-                    const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-                    umma_f16_ss(tmem + sb * 128, make_sdesc_sw128(aQ + off, 16, 1024),
-                                make_sdesc_sw128(kbase + off, 16, 1024), idesc_qk, k > 0);
+                    const uint32_t off = ((k >> 2) * 16384 + (k & 3) * 32) >> 4;
+                    umma_ss_lo(tmem + sb * 128, q_lo + off, kb_lo + off, idesc_qk, k > 0 ? 1u : 0u);
                 }
                 umma_commit(&s_full[sb]);
                 return true;
@@ -303,14 +323,13 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                 if (!mbar_wait(&p_full[g], (t >> 1) & 1, abort_flag)) break;
                 tc_fence_after();
                 const int s = t % FWD_NS;
-                const uint32_t vbase = aV + s * L::TILE;
+                const uint32_t vb_lo = v_lo + uint32_t(s) * (L::TILE >> 4);
                 const uint32_t pbase = tmem + g * 128;
+                const uint32_t acc0 = t >= 2 ? 1u : 0u;
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    umma_f16_ts(tmem + FWD_TMEM_O + g * 128, pbase + k * 8,
-                                make_sdesc_sw128(vbase + k * 2048, 16384, 1024), idesc_pv,
-                                (t >= 2 || k > 0) ? 1u : 0u);
-                }
+                for (int k = 0; k < 8; ++k)
+                    umma_ts_lo(tmem + FWD_TMEM_O + g * 128, pbase + k * 8, vb_lo + k * (2048 >> 4), idesc_pv,
+                               k > 0 ? 1u : acc0);
                 umma_commit(&kv_empty[s]);
                 umma_commit(&pv_done[g]);
             }
@@ -350,15 +369,17 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                 for (int q0 = 0; q0 < 32; q0 += 4) {
                     const float4 g4 = *reinterpret_cast<const float4 *>(gbias + q0);
                     const float gbq[4] = {g4.x, g4.y, g4.z, g4.w};
+                    float v[4];
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const int q = q0 + j, c = q >> 3, i = (q & 7) * 4;
-                        const float gm = fmaxf(fmaxf(__uint_as_float(x[c][i]), __uint_as_float(x[c][i + 1])),
-                                               fmaxf(__uint_as_float(x[c][i + 2]), __uint_as_float(x[c][i + 3])));
-                        const float v = fmaf(gm, p.scale_log2, gbq[j]);
-                        if (j & 1) mt1 = fmaxf(mt1, v);
-                        else mt0 = fmaxf(mt0, v);
+                        const float gm = fmaxf(fmax3(__uint_as_float(x[c][i]), __uint_as_float(x[c][i + 1]),
+                                                     __uint_as_float(x[c][i + 2])),
+                                               __uint_as_float(x[c][i + 3]));
+                        v[j] = fmaf(gm, p.scale_log2, gbq[j]);
                     }
+                    mt0 = fmax3(mt0, v[0], v[1]);
+                    mt1 = fmax3(mt1, v[2], v[3]);
                 }
             } else {
                 const float *bias = sBias + s * 128;
