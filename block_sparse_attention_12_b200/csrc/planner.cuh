@@ -62,7 +62,7 @@ __device__ __forceinline__ void row_uniforms8(uint64_t seed, int64_t b, int64_t 
 
 // vals[j0 .. j0+7] (zero past `end`); two 16-byte shared loads when the
 // eight lie inside the row (j0 is a multiple of 8, so they are aligned).
-__device__ __forceinline__ void load8(const float *vals, int64_t j0, int64_t end, float (&r)[8]) {
+__device__ __forceinline__ void load8(const float *vals, int j0, int end, float (&r)[8]) {
     if (j0 + 8 <= end) {
         const float4 a = *reinterpret_cast<const float4 *>(vals + j0);
         const float4 b = *reinterpret_cast<const float4 *>(vals + j0 + 4);
@@ -143,23 +143,27 @@ __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
     const int64_t row = blockIdx.x;
     const int64_t b = row / (H * nqb), h = (row / nqb) % H, qb = row % nqb;
     const float *src = in + row * nkvb;
-    const int nbytes = int((nkvb + 31) / 32) * 4;
+    int32_t *ridx = idx_out + row * cap;
+    float *rpis = pi_sel + row * cap;
+    const int n = int(nkvb);  // row length (at most kMaxPlanBlocks), 32-bit loop indices below
+    const int ncap_out = int(cap);
+    const int nbytes = ((n + 31) / 32) * 4;
 
     // load (8 independent loads in flight per thread); SIP also counts
     // positive scores and sums them
     int npos_l = 0;
     double sum_l = 0.0;
-    for (int64_t j0 = tid; j0 < nkvb; j0 += 8 * PL_THREADS) {
+    for (int j0 = tid; j0 < n; j0 += 8 * PL_THREADS) {
         float v[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-            const int64_t j = j0 + int64_t(u) * PL_THREADS;
-            v[u] = j < nkvb ? __ldg(src + j) : 0.f;
+            const int j = j0 + u * PL_THREADS;
+            v[u] = j < n ? __ldg(src + j) : 0.f;
         }
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-            const int64_t j = j0 + int64_t(u) * PL_THREADS;
-            if (j < nkvb) {
+            const int j = j0 + u * PL_THREADS;
+            if (j < n) {
                 vals[j] = v[u];
                 if (MODE == kPlanSip) {
                     npos_l += v[u] > 0.f;
@@ -171,14 +175,14 @@ __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
     for (int i = tid; i < nbytes; i += PL_THREADS) flags[i] = 0;
 
     // this warp's segment; lane works on blocks j0 .. j0+7 of each 256-block step
-    const int64_t seg = ((nkvb + PL_WARPS * 256 - 1) / (PL_WARPS * 256)) * 256;
-    const int64_t w0 = int64_t(wid) * seg;
-    const int64_t w1 = w0 + seg < nkvb ? w0 + seg : nkvb;
+    const int seg = ((n + PL_WARPS * 256 - 1) / (PL_WARPS * 256)) * 256;
+    const int w0 = wid * seg;
+    const int w1 = w0 + seg < n ? w0 + seg : n;
 
     if (MODE == kPlanSip) {
         const int npos = block_sum<int>(npos_l, sc.iwarp, &sc.bcast[0]);  // (also orders the loads)
         if (Bblk >= double(npos)) {
-            for (int64_t j = tid; j < nkvb; j += PL_THREADS) vals[j] = vals[j] > 0.f ? 1.f : 0.f;
+            for (int j = tid; j < n; j += PL_THREADS) vals[j] = vals[j] > 0.f ? 1.f : 0.f;
         } else {
             // capping rounds: lambda = (Bblk - |C|) / sum_{j not in C} s_j; C
             // grows by {j : lambda s_j >= 1}, tested exactly in fp64 for the
@@ -188,25 +192,25 @@ __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
             // consecutive blocks form one word, rebuilt by ballot.
             uint32_t *fw = reinterpret_cast<uint32_t *>(flags);
             double rest = block_sum<double>(sum_l, sc.dwarp, &sc.dbcast);
-            int64_t ncap = 0;
+            int ncap = 0;
             double lam = Bblk / rest;
-            for (int64_t round = 0; round <= nkvb; ++round) {
+            for (int round = 0; round <= n; ++round) {
                 const float near = float(lam) * (1.f + 1e-5f);
                 int added_l = 0;
                 double capped_l = 0.0;
                 // four words (128 blocks) per step: four independent chains
-                for (int64_t j128 = w0; j128 < w1; j128 += 128) {
+                for (int j128 = w0; j128 < w1; j128 += 128) {
                     uint32_t word[4];
                     float sv[4];
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        const int64_t j = j128 + 32 * q + lane;
+                        const int j = j128 + 32 * q + lane;
                         word[q] = j128 + 32 * q < w1 ? fw[(j128 >> 5) + q] : 0xFFFFFFFFu;
                         sv[q] = j < w1 ? vals[j] : 0.f;
                     }
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        const int64_t j = j128 + 32 * q + lane;
+                        const int j = j128 + 32 * q + lane;
                         bool cap_now = false;
                         if (j < w1 && !((word[q] >> lane) & 1u) && sv[q] * near >= 1.f &&
                             lam * double(sv[q]) >= 1.0) {
@@ -228,8 +232,8 @@ __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
             }
             // pi into shared memory (lane-strided, conflict-free); the capped
             // flags are cleared again for the sampling pass
-            for (int64_t j32 = w0; j32 < w1; j32 += 32) {
-                const int64_t j = j32 + lane;
+            for (int j32 = w0; j32 < w1; j32 += 32) {
+                const int j = j32 + lane;
                 const uint32_t word = fw[j32 >> 5];
                 if (j < w1) vals[j] = ((word >> lane) & 1u) ? 1.f : __double2float_rn(lam * double(vals[j]));
                 __syncwarp();
@@ -239,7 +243,7 @@ __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
     }
     __syncthreads();
     if (MODE == kPlanSip && pi_out != nullptr)
-        for (int64_t j = tid; j < nkvb; j += PL_THREADS) pi_out[row * nkvb + j] = vals[j];
+        for (int j = tid; j < n; j += PL_THREADS) pi_out[row * nkvb + j] = vals[j];
 
     // top-k threshold: radix select on the fp32 bit patterns of the
     // non-negative scores, 8 bits per pass, most significant first
@@ -251,7 +255,7 @@ __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
         for (int shift = 24; shift >= 0; shift -= 8) {
             for (int i = tid; i < 256; i += PL_THREADS) sc.hist[i] = 0;
             __syncthreads();
-            for (int64_t j = tid; j < nkvb; j += PL_THREADS) {
+            for (int j = tid; j < n; j += PL_THREADS) {
                 const uint32_t bv = __float_as_uint(vals[j]);
                 if ((bv & pmask) == prefix) atomicAdd(&sc.hist[(bv >> shift) & 255u], 1);
             }
@@ -277,14 +281,14 @@ __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
 
     // ---- pass 1: (SIP) final pi; flags <- taken blocks; per-warp counts
     int nsel_w = 0, neq_w = 0;
-    for (int64_t j0 = w0 + 8 * lane; j0 < w1; j0 += 256) {
+    for (int j0 = w0 + 8 * lane; j0 < w1; j0 += 256) {
         uint32_t tk = 0, ek = 0;
         if (MODE == kPlanTopk) {
             float raw[8];
             load8(vals, j0, w1, raw);
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                const int64_t j = j0 + u;
+                const int j = j0 + u;
                 const uint32_t bv = __float_as_uint(raw[u]);
                 tk |= uint32_t(k_top > 0 && j < w1 && bv > thr) << u;
                 ek |= uint32_t(k_top > 0 && j < w1 && bv == thr) << u;
@@ -308,7 +312,7 @@ __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
         sc.wcount2[wid] = neq_w;
     }
     __syncthreads();
-    int64_t pos = 0, eq_rank = 0, total = 0, eq_total = 0;
+    int pos = 0, eq_rank = 0, total = 0, eq_total = 0;
     for (int w = 0; w < PL_WARPS; ++w) {
         if (w < wid) {
             pos += sc.wcount[w];
@@ -324,7 +328,7 @@ __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
     }
 
     // ---- pass 2: compaction in ascending index order within the warp's segment
-    for (int64_t j0 = w0 + 8 * lane; j0 < w1; j0 += 256) {
+    for (int j0 = w0 + 8 * lane; j0 < w1; j0 += 256) {
         uint32_t tk = 0;
         if (MODE == kPlanTopk) {
             uint32_t ek = 0;
@@ -332,7 +336,7 @@ __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
             load8(vals, j0, w1, raw);
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                const int64_t j = j0 + u;
+                const int j = j0 + u;
                 const uint32_t bv = __float_as_uint(raw[u]);
                 tk |= uint32_t(k_top > 0 && j < w1 && bv > thr) << u;
                 ek |= uint32_t(k_top > 0 && j < w1 && bv == thr) << u;
@@ -344,7 +348,7 @@ __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
                 const int y = __shfl_up_sync(0xffffffffu, incl, o);
                 if (lane >= o) incl += y;
             }
-            int64_t r = eq_rank + (incl - neq);  // rank of this lane's first tie
+            int r = eq_rank + (incl - neq);  // rank of this lane's first tie
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 if ((ek >> u) & 1u) {
@@ -363,13 +367,13 @@ __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
             const int y = __shfl_up_sync(0xffffffffu, incl, o);
             if (lane >= o) incl += y;
         }
-        int64_t p = pos + (incl - nt);
+        int p = pos + (incl - nt);
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             if ((tk >> u) & 1u) {
-                if (p < cap) {
-                    idx_out[row * cap + p] = int32_t(j0 + u);
-                    pi_sel[row * cap + p] = MODE == kPlanTopk ? 1.f : vals[j0 + u];
+                if (p < ncap_out) {
+                    ridx[p] = j0 + u;
+                    rpis[p] = MODE == kPlanTopk ? 1.f : vals[j0 + u];
                 }
                 ++p;
             }
@@ -377,8 +381,8 @@ __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
         pos += __shfl_sync(0xffffffffu, incl, 31);
     }
     if (tid == 0) {
-        if (total > cap) raise_error(kErrOverflow);
-        counts[row] = int32_t(total < cap ? total : cap);
+        if (total > ncap_out) raise_error(kErrOverflow);
+        counts[row] = total < ncap_out ? total : ncap_out;
     }
 }
 
