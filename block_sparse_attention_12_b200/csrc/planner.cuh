@@ -21,6 +21,13 @@ namespace abattn {
 
 constexpr int PL_THREADS = 512;
 constexpr int PL_WARPS = PL_THREADS / 32;
+// Capping candidates: blocks left uncapped by the first round whose score is
+// within a factor PL_CAND_ALPHA of that round's threshold.  The later rounds
+// test only these while lambda stays below PL_CAND_ALPHA times its first value
+// (so no other block can reach the threshold); otherwise, or when more than
+// PL_CAND blocks qualify, every round scans the whole row.
+constexpr int PL_CAND = 2048;
+constexpr double PL_CAND_ALPHA = 64.0;
 
 enum PlanMode : int { kPlanSip = 0, kPlanTopk = 1, kPlanFromPi = 2 };
 
@@ -82,6 +89,8 @@ struct PlanScratch {
     int bcast[4];
     double dbcast;
     int hist[256];
+    int ncand;
+    uint16_t cand[PL_CAND];
 };
 
 // Block-wide sums of one int and one double in a single exchange.
@@ -191,11 +200,15 @@ __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
             // walk (conflict-free shared loads); the capped flags of 32
             // consecutive blocks form one word, rebuilt by ballot.
             uint32_t *fw = reinterpret_cast<uint32_t *>(flags);
-            double rest = block_sum<double>(sum_l, sc.dwarp, &sc.dbcast);
+            if (tid == 0) sc.ncand = 0;
+            double rest = block_sum<double>(sum_l, sc.dwarp, &sc.dbcast);  // (also publishes ncand = 0)
             int ncap = 0;
             double lam = Bblk / rest;
-            for (int round = 0; round <= n; ++round) {
+            const double lam_lim = PL_CAND_ALPHA * lam;
+            // one round over the whole row; the first one also collects the candidates
+            auto full_round = [&](bool collect, int &added, double &capped) {
                 const float near = float(lam) * (1.f + 1e-5f);
+                const float cand_near = float(lam_lim) * (1.f + 1e-5f);
                 int added_l = 0;
                 double capped_l = 0.0;
                 // four words (128 blocks) per step: four independent chains
@@ -211,24 +224,60 @@ __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         const int j = j128 + 32 * q + lane;
+                        const bool open = j < w1 && !((word[q] >> lane) & 1u);
                         bool cap_now = false;
-                        if (j < w1 && !((word[q] >> lane) & 1u) && sv[q] * near >= 1.f &&
-                            lam * double(sv[q]) >= 1.0) {
+                        if (open && sv[q] * near >= 1.f && lam * double(sv[q]) >= 1.0) {
                             cap_now = true;
                             ++added_l;
                             capped_l += double(sv[q]);
                         }
                         const uint32_t nb = __ballot_sync(0xffffffffu, cap_now);
                         if (nb != 0u && lane == 0) fw[(j128 >> 5) + q] = word[q] | nb;
+                        if (collect) {
+                            const bool c = open && !cap_now && sv[q] * cand_near >= 1.f;
+                            const uint32_t cm = __ballot_sync(0xffffffffu, c);
+                            if (cm != 0u) {
+                                int base = 0;
+                                if (lane == 0) base = atomicAdd(&sc.ncand, __popc(cm));
+                                base = __shfl_sync(0xffffffffu, base, 0);
+                                const int at = base + __popc(cm & ((1u << lane) - 1u));
+                                if (c && at < PL_CAND) sc.cand[at] = uint16_t(j);
+                            }
+                        }
                     }
                 }
-                int added;
-                double capped;
                 block_sum2(added_l, capped_l, sc, added, capped);
-                if (added == 0) break;
+            };
+            int added;
+            double capped;
+            full_round(true, added, capped);
+            const bool cand_ok = sc.ncand <= PL_CAND;  // read after block_sum2's barriers
+            const int ncand = sc.ncand;
+            bool scan_all = !cand_ok;
+            while (added != 0) {
                 rest -= capped;
                 ncap += added;
                 lam = (Bblk - double(ncap)) / rest;
+                if (lam > lam_lim) scan_all = true;
+                if (scan_all) {
+                    full_round(false, added, capped);
+                } else {
+                    // a round over the candidates only
+                    const float near = float(lam) * (1.f + 1e-5f);
+                    int added_l = 0;
+                    double capped_l = 0.0;
+                    for (int i = tid; i < ncand; i += PL_THREADS) {
+                        const int j = sc.cand[i];
+                        const float sj = vals[j];
+                        const uint32_t bit = 1u << (j & 31);
+                        if (!(fw[j >> 5] & bit) && sj * near >= 1.f && lam * double(sj) >= 1.0) {
+                            atomicOr(&fw[j >> 5], bit);
+                            ++added_l;
+                            capped_l += double(sj);
+                        }
+                    }
+                    block_sum2(added_l, capped_l, sc, added, capped);
+                }
             }
             // pi into shared memory (lane-strided, conflict-free); the capped
             // flags are cleared again for the sampling pass
