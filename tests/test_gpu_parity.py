@@ -208,6 +208,49 @@ def test_waterfill_pi_parity(tiny):
         np.testing.assert_array_equal(pg.counts.cpu().numpy(), po["counts"])
 
 
+def _fallback_rows(n, rng):
+    """Score rows for the water-fill's fallback paths (n = 4096 blocks, 8%
+    budget): (a) lambda grows past 64 times its first value, so the rounds
+    after the first scan the whole row (and cap 100 more blocks); (b) more
+    than 2048 blocks qualify as candidates, so the list overflows and a full
+    round caps 200 more; (c) an ordinary heavy-tailed row (candidate rounds)."""
+    a = np.concatenate([np.full(60, 1e6), np.full(100, 40.0), np.full(n - 160, 1.0)])
+    b = np.concatenate([np.full(60, 2000.0), np.full(200, 500.0), np.full(2100, 12.0), np.full(n - 2360, 0.1)])
+    c = np.exp(rng.standard_normal(n) * 2.0)
+    for r in (a, b):
+        rng.shuffle(r)
+    return [a, b, c]
+
+
+def test_waterfill_fallback_paths():
+    B, H, N, d = 1, 1, 16384, 64
+    cfg = abi.Config(kv_block=4, budget=0.08, seed=11)
+    n = N // 4
+    Bblk = cfg.budget * n
+    rng = np.random.default_rng(5)
+    rows = _fallback_rows(n, rng)
+    # the rows take the paths they are built for
+    lam0 = [Bblk / r.sum() for r in rows]
+    pis = [oracle.waterfill(r, Bblk) for r in rows]
+    assert pis[0][1] / lam0[0] > 64
+    assert ((rows[1] * 64 * lam0[1] >= 1) & (rows[1] * lam0[1] < 1)).sum() > 2048
+    assert (pis[0][0] >= 1).sum() == 160 and (pis[1][0] >= 1).sum() == 260
+    S = np.tile(rows[2], (N // 128, 1))
+    S[:2] = rows[0], rows[1]
+    S32 = torch.from_numpy(S.astype(np.float32)).reshape(B, H, N // 128, n)
+    pg, pig = abi.plan_from_scores(S32.cuda(), (B, H, N, d), cfg, want_pi=True)
+    abi.check()
+    pig = pig.cpu().numpy()[0, 0]
+    counts, idx, ps = (t.cpu().numpy()[0, 0] for t in (pg.counts, pg.idx, pg.pi_sel))
+    for qb in (0, 1, 2, N // 128 - 1):
+        po, _, _ = oracle.waterfill(S32[0, 0, qb].double().numpy(), Bblk)
+        assert np.max(np.abs(pig[qb] - po) / np.maximum(po, 1e-30)) <= 1e-5, qb
+        idx_o, ps_o, n_o = oracle.sample(pig[qb], cfg.seed, 0, 0, qb, pg.cap)
+        assert counts[qb] == min(n_o, pg.cap)
+        np.testing.assert_array_equal(idx[qb, :counts[qb]], idx_o)
+        np.testing.assert_array_equal(ps[qb, :counts[qb]], ps_o)
+
+
 def test_topk_bit_exact_from_fp32_scores(tiny):
     cfg = cfg_of(W, mode=abi.MODE_TOPK)
     shape = tuple(tiny["Q"].shape)
