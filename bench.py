@@ -57,6 +57,11 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--denoise", action="store_true",
+                    help="synthetic denoising loop: dense warm-up steps and first block, a plan every 4 steps")
+    ap.add_argument("--denoise-steps", type=int, default=50)
+    ap.add_argument("--denoise-layers", type=int, default=2)
+    ap.add_argument("--model-layers", type=int, default=40)
     ap.add_argument("--sweep", action="store_true",
                     help="budget x kv_block x (SIP, top-k) sweep on the sweep-75k layer, one JSON line per point")
     return ap.parse_args()
@@ -253,6 +258,27 @@ def timed(fn, iters, stream):
     return e0.elapsed_time(e1) / iters
 
 
+def run_denoise(args):
+    """One JSON line: the denoising-loop policy (first 10 of 50 steps and the
+    first block dense, a plan every 4 steps) over `--denoise-layers` synthetic
+    layers of the workload whose activations drift between steps; attention
+    time per step measured with CUDA events, per-call times solved from it,
+    and the same policy extrapolated to `--model-layers` blocks."""
+    from block_sparse_attention_12_b200 import build, denoise
+    build.build()
+    w = inputs.WORKLOADS[args.workload]
+    if args.heads:
+        import dataclasses
+        w = dataclasses.replace(w, H=args.heads, name=f"{w.name}-{args.heads}heads")
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    pol = denoise.Policy(steps=args.denoise_steps)
+    res = denoise.run(w, pol, layers=args.denoise_layers)
+    dense_ms, sparse_ms, plan_ms = denoise.per_call_ms(pol, res, args.denoise_layers)
+    out = denoise.summary(w, pol, res, args.denoise_layers, dense_ms, sparse_ms, plan_ms, args.model_layers)
+    out["data"] = "synthetic (seeded base + seeded drift per step)"
+    print(json.dumps(out))
+
+
 def run_sweep(args):
     """Budget 5/8/11/25/50/100% x kv_block 4/128 x (SIP, top-k) on the
     75,600-token x 10-head layer: plan and forward time, executed TFLOP/s,
@@ -306,6 +332,9 @@ def main():
     args = parse()
     if args.sweep:
         run_sweep(args)
+        return
+    if args.denoise:
+        run_denoise(args)
         return
     w = inputs.WORKLOADS[args.workload]
     if args.heads:
