@@ -62,6 +62,8 @@ def parse():
     ap.add_argument("--denoise-steps", type=int, default=50)
     ap.add_argument("--denoise-layers", type=int, default=2)
     ap.add_argument("--model-layers", type=int, default=40)
+    ap.add_argument("--strong", action="store_true",
+                    help="one layer's heads sharded over the ranks (head_offset plans, all-gather of O)")
     ap.add_argument("--sweep", action="store_true",
                     help="budget x kv_block x (SIP, top-k) sweep on the sweep-75k layer, one JSON line per point")
     return ap.parse_args()
@@ -258,6 +260,70 @@ def timed(fn, iters, stream):
     return e0.elapsed_time(e1) / iters
 
 
+def run_strong(args):
+    """Strong scaling of one layer: rank r holds heads head_shard(H, r, N),
+    plans them with head_offset = the slice's first head (so the plan equals
+    those rows of the one-GPU plan) and runs the forward; a step ends with the
+    all-gather of O over NCCL.  Timing as in the default mode (barrier and
+    synchronize around K steps, max over ranks); value = the layer's executed
+    TFLOP per step over that time."""
+    from block_sparse_attention_12_b200 import abi, build
+    build.build()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    w = inputs.WORKLOADS[args.workload]
+    hs = multigpu.head_shard(w.H, rank, world)
+    Q, K, V = inputs.make_qkv_heads(w, hs, device=f"cuda:{local}")
+    shape = tuple(Q.shape)
+    cfg = abi.Config(kv_block=w.kv_block, budget=w.budget, n_clusters=w.n_clusters,
+                     kmeans_iters=w.kmeans_iters, seed=w.seed, head_offset=hs.start)
+    planner = abi.Planner(shape, cfg)
+    O = torch.empty_like(Q)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        plan = planner(Q, K)
+        abi.forward(Q, K, V, plan, cfg, O=O, want_lse=False)
+        return multigpu.gather_heads(O, w.H, world)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    abi.check()
+    fl = torch.tensor([abi.executed_flops(planner.plan, shape)], dtype=torch.float64, device=Q.device)
+    if dist:
+        dist.all_reduce(fl)  # the layer's executed FLOP: the ranks' shards summed
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    ms = multigpu.max_over_ranks(e0.elapsed_time(e1) / args.steps, Q.device)
+    abi.check()
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC, "value": float(fl.item()) / (ms / 1e3) / 1e12, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "tokens": w.N, "heads": w.H, "heads_per_rank": len(hs),
+                       "kv_block": w.kv_block, "budget": w.budget,
+                       "step": "abattn_plan + abattn_forward on the rank's heads + all-gather of O",
+                       "parallelism": f"heads sharded over {world} GPUs"},
+        }), flush=True)
+    if dist:
+        dist.destroy_process_group()
+
+
 def run_denoise(args):
     """One JSON line: the denoising-loop policy (first 10 of 50 steps and the
     first block dense, a plan every 4 steps) over `--denoise-layers` synthetic
@@ -335,6 +401,9 @@ def main():
         return
     if args.denoise:
         run_denoise(args)
+        return
+    if args.strong:
+        run_strong(args)
         return
     w = inputs.WORKLOADS[args.workload]
     if args.heads:

@@ -40,7 +40,7 @@ class Params(ctypes.Structure):
     _fields_ = [("q_block", ctypes.c_int32), ("kv_block", ctypes.c_int32),
                 ("n_clusters", ctypes.c_int32), ("kmeans_iters", ctypes.c_int32),
                 ("budget", ctypes.c_float), ("mode", ctypes.c_int32), ("seed", ctypes.c_uint64),
-                ("scale", ctypes.c_float)]
+                ("scale", ctypes.c_float), ("head_offset", ctypes.c_int32)]
 
 
 class AbattnError(RuntimeError):
@@ -120,10 +120,11 @@ class Config:
     seed: int = 0
     scale: float = 0.0
     q_block: int = 128
+    head_offset: int = 0  # global index of the first head when the tensors hold a slice of a layer's heads
 
     def params(self) -> Params:
         return Params(self.q_block, self.kv_block, self.n_clusters, self.kmeans_iters,
-                      float(self.budget), self.mode, self.seed, float(self.scale))
+                      float(self.budget), self.mode, self.seed, float(self.scale), self.head_offset)
 
 
 def dims_of(Q: torch.Tensor) -> Dims:

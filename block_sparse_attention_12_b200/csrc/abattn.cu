@@ -45,6 +45,7 @@ int check_params(const abattn_params *p, bool need_planner) {
     if (p->kmeans_iters < 0 || p->kmeans_iters > 64) return ABATTN_ERR_PARAM;
     if (!(p->budget > 0.f && p->budget <= 1.f)) return ABATTN_ERR_PARAM;
     if (p->mode != ABATTN_MODE_SIP && p->mode != ABATTN_MODE_TOPK) return ABATTN_ERR_PARAM;
+    if (p->head_offset < 0) return ABATTN_ERR_PARAM;
     return ABATTN_OK;
 }
 
@@ -230,17 +231,17 @@ int launch_plan(int mode, const float *in, const abattn_dims *d, const abattn_pa
         case kPlanSip:
             e = cudaFuncSetAttribute(plan_kernel<kPlanSip>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
             if (e != cudaSuccess) return cuda_status(e);
-            plan_kernel<kPlanSip><<<unsigned(rows), PL_THREADS, smem, st>>>(in, d->H, nqb, nkvb, Bblk, k_top, p->seed, cap, counts, idx, pi_sel, pi_out);
+            plan_kernel<kPlanSip><<<unsigned(rows), PL_THREADS, smem, st>>>(in, d->H, p->head_offset, nqb, nkvb, Bblk, k_top, p->seed, cap, counts, idx, pi_sel, pi_out);
             break;
         case kPlanTopk:
             e = cudaFuncSetAttribute(plan_kernel<kPlanTopk>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
             if (e != cudaSuccess) return cuda_status(e);
-            plan_kernel<kPlanTopk><<<unsigned(rows), PL_THREADS, smem, st>>>(in, d->H, nqb, nkvb, Bblk, k_top, p->seed, cap, counts, idx, pi_sel, nullptr);
+            plan_kernel<kPlanTopk><<<unsigned(rows), PL_THREADS, smem, st>>>(in, d->H, p->head_offset, nqb, nkvb, Bblk, k_top, p->seed, cap, counts, idx, pi_sel, nullptr);
             break;
         default:
             e = cudaFuncSetAttribute(plan_kernel<kPlanFromPi>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
             if (e != cudaSuccess) return cuda_status(e);
-            plan_kernel<kPlanFromPi><<<unsigned(rows), PL_THREADS, smem, st>>>(in, d->H, nqb, nkvb, Bblk, k_top, p->seed, cap, counts, idx, pi_sel, nullptr);
+            plan_kernel<kPlanFromPi><<<unsigned(rows), PL_THREADS, smem, st>>>(in, d->H, p->head_offset, nqb, nkvb, Bblk, k_top, p->seed, cap, counts, idx, pi_sel, nullptr);
             break;
     }
     return launch_status();

@@ -141,7 +141,7 @@ __device__ __forceinline__ T block_sum(T v, T *warp_buf, T *bcast) {
 // need a block-wide exchange, so they come out in ascending order.
 template <int MODE>
 __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
-    const float *__restrict__ in, int64_t H, int64_t nqb, int64_t nkvb, double Bblk, int64_t k_top,
+    const float *__restrict__ in, int64_t H, int64_t h_off, int64_t nqb, int64_t nkvb, double Bblk, int64_t k_top,
     uint64_t seed, int64_t cap, int32_t *__restrict__ counts, int32_t *__restrict__ idx_out,
     float *__restrict__ pi_sel, float *__restrict__ pi_out) {
     extern __shared__ float pl_smem[];
@@ -150,7 +150,8 @@ __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
     uint8_t *flags = reinterpret_cast<uint8_t *>(vals + nkvb);               // [ceil(nkvb/32) words]
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int64_t row = blockIdx.x;
-    const int64_t b = row / (H * nqb), h = (row / nqb) % H, qb = row % nqb;
+    // h is the head's global index (the tensors may hold a slice of a layer's heads)
+    const int64_t b = row / (H * nqb), h = (row / nqb) % H + h_off, qb = row % nqb;
     const float *src = in + row * nkvb;
     int32_t *ridx = idx_out + row * cap;
     float *rpis = pi_sel + row * cap;

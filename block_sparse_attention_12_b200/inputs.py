@@ -140,6 +140,20 @@ def make_qkv(w: Workload, device: str = "cpu", seed: int | None = None, threads:
     return Q, K, V
 
 
+def make_qkv_heads(w: Workload, heads: range, device: str = "cpu", seed: int | None = None):
+    """Q, K, V of the heads `heads` of batch 0 only, [1, len(heads), N, d] bf16:
+    the same values as those heads of make_qkv (each head has its own streams)."""
+    seed = w.seed if seed is None else seed
+    pos = (0.8 * position_code(w.grid, w.d)).numpy()
+    rows = outlier_rows(w, seed)
+    Q, K, V = (torch.empty(1, len(heads), w.N, w.d, dtype=torch.bfloat16) for _ in range(3))
+    for i, h in enumerate(heads):
+        Q[0, i], K[0, i], V[0, i] = make_head(w, 0, h, seed, pos, rows)
+    if device != "cpu":
+        Q, K, V = (t.to(device) for t in (Q, K, V))
+    return Q, K, V
+
+
 def row_sample(w: Workload, n_rows: int, seed: int = 1234):
     """A seeded sample of (b, h, qb) rows, used to check large layers."""
     nqb = math.ceil(w.N / w.q_block)

@@ -1,11 +1,16 @@
-"""Host-side plumbing of the multi-GPU benchmark (one process per GPU).
+"""Host-side plumbing of the multi-GPU paths (one process per GPU).
 
 Every (b, h, q-block) row of AB-Attention is independent and the plan's
 uniforms are counter-based on (b, h, q-block, KV block), so the work shards
-across GPUs with no data-path collective: each rank runs whole layers (or
-any subset of heads) on its own GPU and the plan it builds equals the
-corresponding rows of a single-GPU plan.  The only collectives are a
-barrier around the timed region and a max-reduce of the per-rank time.
+across GPUs with no exchange inside the op:
+  * weak scaling: each rank runs whole layers on its own GPU; the only
+    collectives are a barrier around the timed region and a max-reduce of
+    the per-rank time;
+  * head sharding (strong scaling of one layer): each rank holds a
+    contiguous slice of the layer's heads, plans it with the slice's first
+    global head as `head_offset` (so its plan equals those rows of the
+    single-GPU plan) and runs the forward; one all-gather then assembles O
+    on every rank.
 """
 from __future__ import annotations
 
@@ -34,3 +39,23 @@ def head_shard(H: int, rank: int, world: int) -> range:
     base, extra = divmod(H, world)
     lo = rank * base + min(rank, extra)
     return range(lo, lo + base + (1 if rank < extra else 0))
+
+
+def gather_heads(O_local: torch.Tensor, H: int, world: int, group=None) -> torch.Tensor:
+    """All-gather of per-rank head slices [B, h_r, N, d] (the slices of
+    head_shard) into the whole layer's [B, H, N, d] on every rank.  The
+    slices are padded to the largest shard, as an all-gather needs equal
+    sizes."""
+    if world == 1:
+        return O_local
+    B, _, N, d = O_local.shape
+    hmax = -(-H // world)
+    pad = O_local.new_zeros(B, hmax, N, d)
+    pad[:, :O_local.shape[1]] = O_local
+    parts = [torch.empty_like(pad) for _ in range(world)]
+    dist.all_gather(parts, pad, group=group)
+    out = O_local.new_empty(B, H, N, d)
+    for r in range(world):
+        hs = head_shard(H, r, world)
+        out[:, hs.start:hs.stop] = parts[r][:, :len(hs)]
+    return out

@@ -66,6 +66,10 @@ typedef struct {
     int32_t mode;         /* ABATTN_MODE_SIP or ABATTN_MODE_TOPK */
     uint64_t seed;        /* key of the counter-based uniform */
     float scale;          /* softmax scale; 0 means 1/sqrt(d) */
+    int32_t head_offset;  /* global index of these tensors' first head (>= 0): a rank that plans a
+                             slice of a layer's heads passes the slice's first head, so its uniforms,
+                             counter (.., qb, head_offset + h, b), and hence its plan equal those rows
+                             of the whole layer's plan; 0 for a whole layer */
 } abattn_params;
 
 /* Library identification string (static storage). */

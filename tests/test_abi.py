@@ -83,7 +83,7 @@ def test_forward_rejects_null_misaligned_and_capacity(L):
 
 @pytest.mark.parametrize("field,value", [("budget", 0.0), ("budget", 1.5), ("budget", math.nan),
                                          ("n_clusters", 0), ("n_clusters", 9), ("kmeans_iters", -1),
-                                         ("q_block", 64), ("mode", 2)])
+                                         ("q_block", 64), ("mode", 2), ("head_offset", -1)])
 def test_plan_rejects_params(L, field, value):
     d = D(1, 1, 256, 64)
     rc = L.abattn_plan(FAKE, FAKE, ctypes.byref(d), ctypes.byref(params(**{field: value})), FAKE, FAKE, FAKE, 8,
@@ -127,4 +127,5 @@ def test_score_workspace_check(L):
 def test_params_struct_layout_matches_header():
     assert ctypes.sizeof(abi.Params) == 40
     assert abi.Params.seed.offset == 24 and abi.Params.scale.offset == 32
+    assert abi.Params.head_offset.offset == 36
     assert ctypes.sizeof(abi.Dims) == 32

@@ -251,6 +251,36 @@ def test_waterfill_fallback_paths():
         np.testing.assert_array_equal(ps[qb, :counts[qb]], ps_o)
 
 
+def test_head_offset_slices_equal_whole_layer(tiny):
+    """A rank holding a slice of the heads plans it with head_offset = the
+    slice's first global head: its plan and output equal those rows of the
+    whole layer's (bit for bit), and without the offset the plan differs."""
+    cfg = cfg_of(W)
+    full = abi.plan(tiny["Q"], tiny["K"], cfg)
+    Of, lf = abi.forward(tiny["Q"], tiny["K"], tiny["V"], full, cfg)
+    n_full = full.counts.cpu().numpy()
+    for lo in range(W.H):
+        Qs, Ks, Vs = (t[:, lo:lo + 1].contiguous() for t in (tiny["Q"], tiny["K"], tiny["V"]))
+        cs = cfg_of(W, head_offset=lo)
+        ps = abi.plan(Qs, Ks, cs)
+        Os, ls = abi.forward(Qs, Ks, Vs, ps, cs)
+        abi.check()
+        n = ps.counts.cpu().numpy()
+        np.testing.assert_array_equal(n[0, 0], n_full[0, lo])
+        for qb in range(n.shape[2]):
+            c = n[0, 0, qb]
+            assert torch.equal(ps.idx[0, 0, qb, :c], full.idx[0, lo, qb, :c])
+            assert torch.equal(ps.pi_sel[0, 0, qb, :c], full.pi_sel[0, lo, qb, :c])
+        assert torch.equal(Os[0, 0], Of[0, lo]) and torch.equal(ls[0, 0], lf[0, lo])
+    # head 1 planned as if it were head 0 draws other uniforms
+    p0 = abi.plan(tiny["Q"][:, 1:2].contiguous(), tiny["K"][:, 1:2].contiguous(), cfg_of(W))
+    abi.check()
+    differs = any(not torch.equal(p0.idx[0, 0, qb, :int(p0.counts[0, 0, qb])],
+                                  full.idx[0, 1, qb, :int(full.counts[0, 1, qb])])
+                  for qb in range(p0.counts.shape[2]))
+    assert differs
+
+
 def test_topk_bit_exact_from_fp32_scores(tiny):
     cfg = cfg_of(W, mode=abi.MODE_TOPK)
     shape = tuple(tiny["Q"].shape)

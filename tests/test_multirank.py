@@ -62,9 +62,22 @@ def _plan_worker(rank, world, port, out):
         dist.destroy_process_group()
 
 
+def _gather_worker(rank, world, port, out):
+    _init(rank, world, port)
+    try:
+        H = 5
+        hs = multigpu.head_shard(H, rank, world)
+        # each rank's slice holds its global head indices
+        O = torch.arange(hs.start, hs.stop, dtype=torch.float32).view(1, -1, 1, 1).expand(1, len(hs), 3, 2).contiguous()
+        full = multigpu.gather_heads(O, H, world)
+        out[rank] = full.numpy()
+    finally:
+        dist.destroy_process_group()
+
+
 def _run(fn, world):
     port = 29500 + (os.getpid() % 1000)
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.spawn(fn, args=(world, port, out), nprocs=world, join=True)
         return dict(out)
@@ -95,3 +108,17 @@ def test_sharded_plan_equals_single_process_plan():
         h, qb, n = int(row[0]), int(row[1]), int(row[2])
         assert full["counts"][0, h, qb] == n
         np.testing.assert_array_equal(row[3:3 + n], full["idx"][0, h, qb, :n])
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_gather_heads_assembles_the_layer(world):
+    out = _run(_gather_worker, world)
+    want = np.arange(5, dtype=np.float32).reshape(1, 5, 1, 1) * np.ones((1, 5, 3, 2), dtype=np.float32)
+    for r in range(world):
+        np.testing.assert_array_equal(out[r], want)
+
+
+def test_head_slice_inputs_equal_the_layer():
+    Q, K, V = inputs.make_qkv(W)
+    Qs, Ks, Vs = inputs.make_qkv_heads(W, range(1, 2))
+    assert torch.equal(Qs, Q[:, 1:2]) and torch.equal(Ks, K[:, 1:2]) and torch.equal(Vs, V[:, 1:2])
