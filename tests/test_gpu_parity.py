@@ -350,7 +350,9 @@ def test_full_plan_equals_dense(tiny):
 # N % 4 == 0 takes the kernel's per-group bias path, the rest its per-key path
 @pytest.mark.parametrize("d,N,kb,budget", [(128, 1000, 4, 0.2), (128, 300, 128, 0.5), (64, 777, 128, 1.0),
                                            (128, 640, 16, 0.3), (64, 2048, 8, 0.1), (128, 1234, 4, 0.25),
-                                           (64, 1003, 32, 0.4)])
+                                           (64, 1003, 32, 0.4),
+                                           # degenerate: one query and one block, a few keys, one tile + 2
+                                           (64, 1, 4, 1.0), (128, 5, 4, 0.5), (128, 130, 4, 0.3)])
 def test_sparse_forward_ragged_shapes(d, N, kb, budget):
     g = torch.Generator().manual_seed(N + kb)
     Qc, Kc, Vc = (torch.randn(1, 2, N, d, generator=g).to(torch.bfloat16) for _ in range(3))
