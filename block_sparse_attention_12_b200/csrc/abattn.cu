@@ -282,6 +282,8 @@ int run_forward(bool dense, const void *Q, const void *K, const void *V, const a
     if ((rc = make_map(&mQ, Q, d, 128)) || (rc = make_map(&mK, K, d, box)) || (rc = make_map(&mV, V, d, box)))
         return rc;
     FwdParams fp;
+    fp.K = static_cast<const __nv_bfloat16 *>(K);
+    fp.V = static_cast<const __nv_bfloat16 *>(V);
     fp.counts = counts;
     fp.idx = idx;
     fp.pi_sel = pi_sel;

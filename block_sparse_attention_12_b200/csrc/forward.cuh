@@ -15,19 +15,18 @@
 //               and hide each other's latencies.  One query row per thread
 //               (TMEM lane); logits t = s * scale * log2(e) + log2(1/pi);
 //               running max with lazy O rescaling (only when the max grows by
-//               more than 2^8); P = exp2(t - m) packed to bf16 and stored back
-//               to TMEM over the first 64 columns of its S buffer.  At the end
-//               the two partial softmaxes are merged (max, sums, O) and O
-//               (bf16) and the natural-log LSE are written;
+//               more than 2^32); P = exp2(t - m), packed to bf16 as it is
+//               computed and stored back to TMEM over the first 64 columns of
+//               its S buffer.  At the end the two partial softmaxes are merged
+//               (max, sums, O) and O (bf16) and the natural-log LSE are written;
 //   warps 8..11, 13..15  producers (setmaxnreg lowered): warp 8 loads the Q
-//               tile once; a 128-key tile is cut into units of R = min(kb, 32)
-//               keys and producer w (0..6) owns units w, w+7, ...: per unit
-//               one TMA box of R rows per 64-column half, for K and for V
-//               (128-byte swizzle, 3 stages), and the bias log2(1/pi) of its R
-//               keys.  Each lane owns one unit and prefetches the next tile's
-//               plan entries.  Small boxes cost the issuing warp tens of cycles
-//               each, so the 128 boxes of a 4-token tile are spread over seven
-//               warps;
+//               tile once by TMA.  Sparse kernel: the 32 quads of 4 rows of a
+//               128-key tile are gathered with cp.async, 16 bytes per lane,
+//               into the 128-byte-swizzled layout (warp w takes quads w,
+//               w+7, ...), with the bias log2(1/pi) of each quad; dense kernel:
+//               one TMA box of 32 rows per 64-column half and tensor.  K and V
+//               share a ring of 3 stages.  The lanes prefetch the plan entries
+//               two tiles ahead;
 //   warp 12     TMEM owner and MMA issuer (setmaxnreg lowered): S = Q K^T
 //               (both operands in shared memory) into S buffer t % 2;
 //               O_{t%2} += P V with P read from TMEM and V from shared memory;
@@ -58,10 +57,20 @@ static_assert(2 * 128 * FWD_SOFTMAX_REGS + 2 * 128 * FWD_OTHER_REGS <= FWD_THREA
               "setmaxnreg split exceeds the launch register budget");
 constexpr int FWD_PRODUCERS = 7;  // producer warps (8..11, 13..15); warp w owns the tile's block slots = w mod 7
 constexpr int FWD_NS = 3;  // K/V stages
+// O and the row sum are rescaled only when a tile's max exceeds the running
+// reference max by more than this (log2 units).  Probabilities then stay
+// below 2^FWD_RESCALE_LOG2, so O <= keys * 2^32 * max|V| and l stay far
+// inside the fp32 range, and bf16 P keeps its relative precision.
+#ifndef ABATTN_FWD_RESCALE_LOG2
+#define ABATTN_FWD_RESCALE_LOG2 32
+#endif
+constexpr float FWD_RESCALE_LOG2 = ABATTN_FWD_RESCALE_LOG2;
 constexpr uint32_t FWD_TMEM_COLS = 512;
 constexpr uint32_t FWD_TMEM_O = 256;  // O accumulators: even tiles at 256, odd tiles at 384
 
 struct FwdParams {
+    const __nv_bfloat16 *K;  // [B*H][N][HD], gathered by the sparse kernel
+    const __nv_bfloat16 *V;
     const int32_t *counts;
     const int32_t *idx;
     const float *pi_sel;
@@ -143,7 +152,10 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
         for (int s = 0; s < FWD_NS; ++s) {
-            mbar_init(&kv_full[s], FWD_PRODUCERS);
+            // dense: one expect_tx arrival per producer warp (TMA bytes);
+            // sparse: one cp.async completion arrival per producer thread plus
+            // one release arrival per warp for the biases
+            mbar_init(&kv_full[s], DENSE ? FWD_PRODUCERS : FWD_PRODUCERS * 33);
             mbar_init(&kv_empty[s], 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -182,113 +194,151 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
             const int32_t *ridx = DENSE ? nullptr : p.idx + int64_t(row) * p.cap;
             const float *rpi = DENSE ? nullptr : p.pi_sel + int64_t(row) * p.cap;
             const int kb = p.kb;                      // rows per block (128 for the dense kernel)
-            const int R = p.box_rows;                 // rows per TMA box: min(kb, 32)
             const int spt = 128 / kb;                 // block slots per tile
-            const int nunits = 128 / R;               // boxes (units) per tile and tensor half
-            const int unit = pw + FWD_PRODUCERS * lane;  // this lane's unit in every tile
-            const bool owner = unit < nunits;
-            const int sl = owner ? (unit * R) / kb : 0;  // the unit's block slot in the tile
-            const int ro = (unit * R) % kb;           // the unit's first row inside its block
-            // units owned by this warp in a tile: those congruent to pw modulo FWD_PRODUCERS
-            const int nown = nunits > pw ? (nunits - pw + FWD_PRODUCERS - 1) / FWD_PRODUCERS : 0;
-            const uint32_t tx_bytes = uint32_t(nown) * R * HD * 2 * 2;
-            int fill_blk = 0;                         // a valid block to load into padding slots
-            if (!DENSE) {
-                const int b0 = ridx[0];
-                fill_blk = (b0 >= 0 && b0 < p.nkvb) ? b0 : 0;
-            }
-            auto fetch = [&](int t, int &blk, float &pi) {
-                const int e = t * spt + sl;
-                blk = -1;
-                pi = 0.f;
-                if (!DENSE && owner && e < cnt) {
-                    blk = __ldg(ridx + e);
-                    pi = __ldg(rpi + e);
-                }
-            };
-            if (!DENSE) {
-                // the plan row is read once per tile by every producer lane:
-                // bring it into L1 up front
-                const int lines = (cnt * 4 + 127) / 128;
-                for (int i = pw * 32 + lane; i < 2 * lines; i += FWD_PRODUCERS * 32)
-                    prefetch_l1(i < lines ? reinterpret_cast<const char *>(ridx) + i * 128
-                                          : reinterpret_cast<const char *>(rpi) + (i - lines) * 128);
-            }
-            // plan entries of tiles t (cur) and t+1 (nxt); the entry of tile
-            // t+2 is fetched at the top of iteration t
-            int cur_blk, nxt_blk;
-            float cur_pi, nxt_pi;
-            fetch(0, cur_blk, cur_pi);
-            fetch(1, nxt_blk, nxt_pi);
-            for (int t = 0; t < T; ++t) {
-                const int s = t % FWD_NS;
-                int x_blk;
-                float x_pi;
-                fetch(t + 2, x_blk, x_pi);
-                if (t >= FWD_NS && !mbar_wait(&kv_empty[s], ((t / FWD_NS) - 1) & 1, abort_flag)) break;
-                int key0 = 0;
-                if (owner) {
-                    // block of this unit, its validity and the bias of its R keys
-                    int blk;
-                    float b = -INFINITY;
-                    if (DENSE) {
-                        blk = t;
-                        b = 0.f;
-                    } else if (t * spt + sl < cnt) {
-                        const bool ok_blk = cur_blk >= 0 && cur_blk < p.nkvb && cur_pi > 0.f;
-                        if (ok_blk) {
-                            blk = cur_blk;
-                            b = -log2f(cur_pi);
+            if constexpr (DENSE) {
+                // whole 128-key tiles: units of R = 32 rows, one TMA box per
+                // unit, 64-column half and tensor
+                const int R = p.box_rows;
+                const int nunits = 128 / R;
+                const int unit = pw + FWD_PRODUCERS * lane;  // this lane's unit in every tile
+                const bool owner = unit < nunits;
+                const int ro = (unit * R) % kb;       // the unit's first row inside its tile
+                const int nown = nunits > pw ? (nunits - pw + FWD_PRODUCERS - 1) / FWD_PRODUCERS : 0;
+                const uint32_t tx_bytes = uint32_t(nown) * R * HD * 2 * 2;
+                for (int t = 0; t < T; ++t) {
+                    const int s = t % FWD_NS;
+                    if (t >= FWD_NS && !mbar_wait(&kv_empty[s], ((t / FWD_NS) - 1) & 1, abort_flag)) break;
+                    if (owner) {
+                        const int key0 = t * kb + ro;
+                        if constexpr (GROUPED) {
+                            float *gdst = sGBias + s * 32 + unit * (R / 4);
+                            for (int i = 0; i < R; i += 4) gdst[i / 4] = key0 + i < p.N ? 0.f : -INFINITY;
                         } else {
-                            blk = fill_blk;
-                            if (ro == 0) raise_error(kErrBounds);
+                            float *bdst = sBias + s * 128 + unit * R;
+                            for (int i = 0; i < R; ++i) bdst[i] = key0 + i < p.N ? 0.f : -INFINITY;
                         }
-                    } else {
-                        blk = fill_blk;  // padding slot: loaded, weighted zero
-                    }
-                    key0 = blk * kb + ro;
-                    if constexpr (GROUPED) {
-                        // scalar stores: a unit's groups start at a multiple of R / 4
-                        // floats, which is 16-byte aligned only for R >= 16
-                        float *gdst = sGBias + s * 32 + unit * (R / 4);
-                        for (int i = 0; i < R; i += 4) gdst[i / 4] = key0 + i < p.N ? b : -INFINITY;
-                    } else {
-                        float *bdst = sBias + s * 128 + unit * R;
-                        for (int i = 0; i < R; i += 4) {
-                            float4 v;
-                            v.x = key0 + i + 0 < p.N ? b : -INFINITY;
-                            v.y = key0 + i + 1 < p.N ? b : -INFINITY;
-                            v.z = key0 + i + 2 < p.N ? b : -INFINITY;
-                            v.w = key0 + i + 3 < p.N ? b : -INFINITY;
-                            *reinterpret_cast<float4 *>(bdst + i) = v;
-                        }
-                    }
-                    __syncwarp(__activemask());
-                    if (lane == 0) mbar_arrive_expect_tx(&kv_full[s], tx_bytes);
-                    __syncwarp(__activemask());
-                    uint8_t *dK = sK + s * L::TILE + unit * R * 128;
-                    uint8_t *dV = sV + s * L::TILE + unit * R * 128;
+                        __syncwarp(__activemask());
+                        if (lane == 0) mbar_arrive_expect_tx(&kv_full[s], tx_bytes);
+                        __syncwarp(__activemask());
+                        uint8_t *dK = sK + s * L::TILE + unit * R * 128;
+                        uint8_t *dV = sV + s * L::TILE + unit * R * 128;
 #pragma unroll
-                    for (int h = 0; h < L::HALVES; ++h) {
-                        tma_load_3d(dK + h * 16384, &tmK, &kv_full[s], h * 64, key0, bh);
-                        tma_load_3d(dV + h * 16384, &tmV, &kv_full[s], h * 64, key0, bh);
+                        for (int h = 0; h < L::HALVES; ++h) {
+                            tma_load_3d(dK + h * 16384, &tmK, &kv_full[s], h * 64, key0, bh);
+                            tma_load_3d(dV + h * 16384, &tmV, &kv_full[s], h * 64, key0, bh);
+                        }
+                    } else if (lane == 0) {
+                        mbar_arrive_expect_tx(&kv_full[s], 0);  // a warp without units still arrives
                     }
-                } else if (lane == 0) {
-                    mbar_arrive_expect_tx(&kv_full[s], 0);  // a warp without units still arrives
+                    __syncwarp();
+                    ++issued;
                 }
-                __syncwarp();
-                cur_blk = nxt_blk;
-                cur_pi = nxt_pi;
-                nxt_blk = x_blk;
-                nxt_pi = x_pi;
-                ++issued;
+            } else {
+                // Selected blocks: the tile's 32 quads of 4 rows (a quad lies in
+                // one block since kb >= 4); warp pw gathers quads pw, pw+7, ...
+                // with cp.async, 16 bytes per lane (row r = lane / 8 of the quad,
+                // chunk c = lane % 8 of a 64-column half), written straight into
+                // the 128-byte-swizzled layout the MMAs read.  Small TMA boxes
+                // would cost the issuing warps tens of cycles each (128 per
+                // tile); cp.async issues one warp instruction per quad, half and
+                // tensor.  kv_full counts one completion arrival per producer
+                // thread (cp.async.mbarrier.arrive.noinc) and one release
+                // arrival per warp after its bias stores.
+                const int nown = (32 - pw + FWD_PRODUCERS - 1) / FWD_PRODUCERS;  // quads of this warp
+                const bool owner = lane < nown;       // lane j fetches the plan entry of quad pw + 7j
+                const int my_q = pw + FWD_PRODUCERS * lane;
+                const int sl = owner ? (my_q * 4) / kb : 0;  // the quad's block slot in the tile
+                const int ro = owner ? (my_q * 4) % kb : 0;  // the quad's first row inside its block
+                const int r = lane >> 3, c = lane & 7;
+                const __nv_bfloat16 *Kbh = p.K + int64_t(bh) * p.N * HD;
+                const __nv_bfloat16 *Vbh = p.V + int64_t(bh) * p.N * HD;
+                int fill_blk = 0;                     // a valid block to load into padding slots
+                {
+                    const int b0 = ridx[0];
+                    fill_blk = (b0 >= 0 && b0 < p.nkvb) ? b0 : 0;
+                }
+                auto fetch = [&](int t, int &blk, float &pi) {
+                    const int e = t * spt + sl;
+                    blk = -1;
+                    pi = 0.f;
+                    if (owner && e < cnt) {
+                        blk = __ldg(ridx + e);
+                        pi = __ldg(rpi + e);
+                    }
+                };
+                {
+                    // the plan row is read once per tile by the producer lanes:
+                    // bring it into L1 up front
+                    const int lines = (cnt * 4 + 127) / 128;
+                    for (int i = pw * 32 + lane; i < 2 * lines; i += FWD_PRODUCERS * 32)
+                        prefetch_l1(i < lines ? reinterpret_cast<const char *>(ridx) + i * 128
+                                              : reinterpret_cast<const char *>(rpi) + (i - lines) * 128);
+                }
+                // plan entries of tiles t (cur) and t+1 (nxt); the entry of tile
+                // t+2 is fetched at the top of iteration t
+                int cur_blk, nxt_blk;
+                float cur_pi, nxt_pi;
+                fetch(0, cur_blk, cur_pi);
+                fetch(1, nxt_blk, nxt_pi);
+                for (int t = 0; t < T; ++t) {
+                    const int s = t % FWD_NS;
+                    int x_blk;
+                    float x_pi;
+                    fetch(t + 2, x_blk, x_pi);
+                    if (t >= FWD_NS && !mbar_wait(&kv_empty[s], ((t / FWD_NS) - 1) & 1, abort_flag)) break;
+                    // this lane's quad: block, first key and bias
+                    int key0 = 0;
+                    float b = -INFINITY;
+                    if (owner) {
+                        int blk = fill_blk;  // padding slot: loaded, weighted zero
+                        if (t * spt + sl < cnt) {
+                            if (cur_blk >= 0 && cur_blk < p.nkvb && cur_pi > 0.f) {
+                                blk = cur_blk;
+                                b = -log2f(cur_pi);
+                            } else if (ro == 0) {
+                                raise_error(kErrBounds);
+                            }
+                        }
+                        key0 = blk * kb + ro;
+                    }
+                    for (int j = 0; j < nown; ++j) {
+                        const int q = pw + FWD_PRODUCERS * j;
+                        const int k0 = __shfl_sync(0xffffffffu, key0, j);
+                        const float bj = __shfl_sync(0xffffffffu, b, j);
+                        const int key = k0 + r;
+                        const bool valid = key < p.N;  // rows past N (ragged last block) read as zero
+                        const int srow = q * 4 + r;
+                        const uint32_t soff = uint32_t(s * L::TILE + srow * 128 + ((c ^ (srow & 7)) << 4));
+                        const int64_t goff = int64_t(valid ? key : 0) * HD + c * 8;
+#pragma unroll
+                        for (int h = 0; h < L::HALVES; ++h) {
+                            cp_async16(sK + soff + h * 16384, Kbh + goff + h * 64, valid);
+                            cp_async16(sV + soff + h * 16384, Vbh + goff + h * 64, valid);
+                        }
+                        if constexpr (GROUPED) {
+                            if (lane == 0) sGBias[s * 32 + q] = k0 < p.N ? bj : -INFINITY;
+                        } else {
+                            if (c == 0) sBias[s * 128 + q * 4 + r] = valid ? bj : -INFINITY;
+                        }
+                    }
+                    cp_async_mbar_arrive_noinc(&kv_full[s]);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&kv_full[s]);
+                    cur_blk = nxt_blk;
+                    cur_pi = nxt_pi;
+                    nxt_blk = x_blk;
+                    nxt_pi = x_pi;
+                    ++issued;
+                }
+                cp_async_wait_all();
             }
             // drain: every issued copy lands before the CTA may exit
             if (*abort_flag) {
                 if (lane == 0) {
                     if (pw == 0) mbar_drain(q_full, 0);
-                    for (int t = issued - FWD_NS < 0 ? 0 : issued - FWD_NS; t < issued; ++t)
-                        mbar_drain(&kv_full[t % FWD_NS], (t / FWD_NS) & 1);
+                    if (DENSE)
+                        for (int t = issued - FWD_NS < 0 ? 0 : issued - FWD_NS; t < issued; ++t)
+                            mbar_drain(&kv_full[t % FWD_NS], (t / FWD_NS) & 1);
                 }
             }
         }
@@ -306,6 +356,10 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
             auto issue_qk = [&](int t) -> bool {
                 const int s = t % FWD_NS, sb = t & 1;
                 if (!mbar_wait(&kv_full[s], (t / FWD_NS) & 1, abort_flag)) return false;
+                // the sparse tile was written by cp.async (generic proxy): order
+                // those writes, observed through the barrier, before the MMAs'
+                // async-proxy reads
+                if (!DENSE) fence_proxy_async_smem();
                 tc_fence_after();
                 const uint32_t kb_lo = k_lo + uint32_t(s) * (L::TILE >> 4);
 #pragma unroll
@@ -355,54 +409,109 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                 break;
             }
             tc_fence_after();
-            uint32_t x[4][32];
+            uint32_t x[4][32];  // the S row
 #pragma unroll
             for (int c = 0; c < 4; ++c) tmem_ld32(t_S + c * 32, x[c]);
             tmem_wait_ld();
-
-            float mt0 = -INFINITY, mt1 = -INFINITY;
             const float *gbias = sGBias + s * 32;
-            if constexpr (GROUPED) {
-                // one bias per group of 4 keys (scale > 0): the row max is taken on
-                // the raw group maxima, one FFMA per group
+            const float *bias = sBias + s * 128;
+            const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+            float2 rs01 = make_float2(0.f, 0.f), rs23 = make_float2(0.f, 0.f);
+            // P as packed bf16 pairs: column j of the row holds keys 2j, 2j+1
+            uint32_t pk[64];
+            // 2^(a*mul + off) for the four keys of group q (two packed pairs):
+            // packed FFMA for the logit shift, SFU exponentials, packed adds
+            // into the row sum, bf16 packing into pk
+            auto exp_group = [&](int q, float2 a, float2 b, float2 mul2, float2 off_a, float2 off_b) {
+                a = __ffma2_rn(a, mul2, off_a);
+                b = __ffma2_rn(b, mul2, off_b);
+                a = make_float2(fast_exp2(a.x), fast_exp2(a.y));
+                b = make_float2(fast_exp2(b.x), fast_exp2(b.y));
+                rs01 = __fadd2_rn(rs01, a);
+                rs23 = __fadd2_rn(rs23, b);
+                pk[2 * q] = pack_bf16x2(a.x, a.y);
+                pk[2 * q + 1] = pack_bf16x2(b.x, b.y);
+            };
+            auto xa = [&](int q) {
+                const int c = q >> 3, i = (q & 7) * 4;
+                return make_float2(__uint_as_float(x[c][i]), __uint_as_float(x[c][i + 1]));
+            };
+            auto xb = [&](int q) {
+                const int c = q >> 3, i = (q & 7) * 4;
+                return make_float2(__uint_as_float(x[c][i + 2]), __uint_as_float(x[c][i + 3]));
+            };
+            // largest raw logit of group q
+            auto gmax = [&](int q) {
+                const int c = q >> 3, i = (q & 7) * 4;
+                return fmaxf(fmax3(__uint_as_float(x[c][i]), __uint_as_float(x[c][i + 1]),
+                                   __uint_as_float(x[c][i + 2])),
+                             __uint_as_float(x[c][i + 3]));
+            };
+            // The tile's largest biased logit.  With GROUPED it is taken on the raw
+            // group maxima (scale > 0), one FFMA per group; otherwise per key,
+            // and x then holds the biased logits.
+            auto max_pass = [&]() -> float {
+                float mt0 = -INFINITY, mt1 = -INFINITY;
 #pragma unroll
                 for (int q0 = 0; q0 < 32; q0 += 4) {
-                    const float4 g4 = *reinterpret_cast<const float4 *>(gbias + q0);
-                    const float gbq[4] = {g4.x, g4.y, g4.z, g4.w};
-                    float v[4];
+                    if constexpr (GROUPED) {
+                        const float4 g4 = *reinterpret_cast<const float4 *>(gbias + q0);
+                        float gm[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) gm[j] = gmax(q0 + j);
+                        const float2 v01 = __ffma2_rn(make_float2(gm[0], gm[1]), sc2, make_float2(g4.x, g4.y));
+                        const float2 v23 = __ffma2_rn(make_float2(gm[2], gm[3]), sc2, make_float2(g4.z, g4.w));
+                        mt0 = fmax3(mt0, v01.x, v01.y);
+                        mt1 = fmax3(mt1, v23.x, v23.y);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int q = q0 + j;
+                            const float4 bb = *reinterpret_cast<const float4 *>(bias + 4 * q);
+                            const float2 va = __ffma2_rn(xa(q), sc2, make_float2(bb.x, bb.y));
+                            const float2 vb = __ffma2_rn(xb(q), sc2, make_float2(bb.z, bb.w));
+                            mt0 = fmax3(mt0, va.x, va.y);
+                            mt1 = fmax3(mt1, vb.x, vb.y);
+                            // keep the biased logit for the exponentials
+                            const int c = q >> 3, i = (q & 7) * 4;
+                            x[c][i + 0] = __float_as_uint(va.x);
+                            x[c][i + 1] = __float_as_uint(va.y);
+                            x[c][i + 2] = __float_as_uint(vb.x);
+                            x[c][i + 3] = __float_as_uint(vb.y);
+                        }
+                    }
+                }
+                return fmaxf(mt0, mt1);
+            };
+            // P = 2^(logit - m_ref) into pk, and the row sum
+            auto exp_pass = [&](float m_ref) {
+#pragma unroll
+                for (int q0 = 0; q0 < 32; q0 += 4) {
+                    float4 g4;
+                    if constexpr (GROUPED) g4 = *reinterpret_cast<const float4 *>(gbias + q0);
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
-                        const int q = q0 + j, c = q >> 3, i = (q & 7) * 4;
-                        const float gm = fmaxf(fmax3(__uint_as_float(x[c][i]), __uint_as_float(x[c][i + 1]),
-                                                     __uint_as_float(x[c][i + 2])),
-                                               __uint_as_float(x[c][i + 3]));
-                        v[j] = fmaf(gm, p.scale_log2, gbq[j]);
-                    }
-                    mt0 = fmax3(mt0, v[0], v[1]);
-                    mt1 = fmax3(mt1, v[2], v[3]);
-                }
-            } else {
-                const float *bias = sBias + s * 128;
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-#pragma unroll
-                    for (int i = 0; i < 32; i += 4) {
-                        const float4 bb = *reinterpret_cast<const float4 *>(bias + c * 32 + i);
-                        const float v0 = fmaf(__uint_as_float(x[c][i + 0]), p.scale_log2, bb.x);
-                        const float v1 = fmaf(__uint_as_float(x[c][i + 1]), p.scale_log2, bb.y);
-                        const float v2 = fmaf(__uint_as_float(x[c][i + 2]), p.scale_log2, bb.z);
-                        const float v3 = fmaf(__uint_as_float(x[c][i + 3]), p.scale_log2, bb.w);
-                        x[c][i + 0] = __float_as_uint(v0);
-                        x[c][i + 1] = __float_as_uint(v1);
-                        x[c][i + 2] = __float_as_uint(v2);
-                        x[c][i + 3] = __float_as_uint(v3);
-                        mt0 = fmaxf(mt0, fmaxf(v0, v1));
-                        mt1 = fmaxf(mt1, fmaxf(v2, v3));
+                        const int q = q0 + j;
+                        if constexpr (GROUPED) {
+                            const float gb = j == 0 ? g4.x : j == 1 ? g4.y : j == 2 ? g4.z : g4.w;
+                            const float2 off = make_float2(gb - m_ref, gb - m_ref);
+                            exp_group(q, xa(q), xb(q), sc2, off, off);
+                        } else {
+                            const float2 neg_m = make_float2(-m_ref, -m_ref);
+                            exp_group(q, xa(q), xb(q), make_float2(1.f, 1.f), neg_m, neg_m);
+                        }
                     }
                 }
-            }
-            const float m_new = fmaxf(m, fmaxf(mt0, mt1));
-            const bool need = m_new > m + 8.f;
+            };
+            // P row -> TMEM over the first 64 columns of this S buffer
+            auto store_p = [&]() {
+                tmem_st32(t_S, *reinterpret_cast<const uint32_t(*)[32]>(pk));
+                tmem_st32(t_S + 32, *reinterpret_cast<const uint32_t(*)[32]>(pk + 32));
+            };
+            // Lazy rescaling: O and l keep the reference max m until a tile's
+            // max exceeds it by more than FWD_RESCALE_LOG2.
+            const float m_new = fmaxf(m, max_pass());
+            const bool need = m_new > m + FWD_RESCALE_LOG2;
             float alpha = 1.f;
             if (need) {
                 alpha = fast_exp2(m - m_new);
@@ -410,48 +519,9 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                 m = m_new;
             }
             const bool any = __any_sync(0xffffffffu, need);
-            const float m_use = (m == -INFINITY) ? 0.f : m;
-            float rs[4] = {0.f, 0.f, 0.f, 0.f};
-            if constexpr (GROUPED) {
-#pragma unroll
-                for (int q0 = 0; q0 < 32; q0 += 4) {
-                    const float4 g4 = *reinterpret_cast<const float4 *>(gbias + q0);
-                    const float gbq[4] = {g4.x, g4.y, g4.z, g4.w};
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int q = q0 + j, c = q >> 3, i = (q & 7) * 4;
-                        const float off = gbq[j] - m_use;
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const float e = fast_exp2(fmaf(__uint_as_float(x[c][i + k]), p.scale_log2, off));
-                            rs[k] += e;
-                            x[c][i + k] = __float_as_uint(e);
-                        }
-                    }
-                }
-            } else {
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const float e = fast_exp2(__uint_as_float(x[c][i]) - m_use);
-                        rs[i & 3] += e;
-                        x[c][i] = __float_as_uint(e);
-                    }
-                }
-            }
-            l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
-            // P row -> TMEM, packed bf16 pairs over the first 64 columns of this S buffer
-#pragma unroll
-            for (int c = 0; c < 4; c += 2) {
-                uint32_t pk[32];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    pk[i] = pack_bf16x2(__uint_as_float(x[c][2 * i]), __uint_as_float(x[c][2 * i + 1]));
-                    pk[16 + i] = pack_bf16x2(__uint_as_float(x[c + 1][2 * i]), __uint_as_float(x[c + 1][2 * i + 1]));
-                }
-                tmem_st32(t_S + c * 16, pk);
-            }
+            exp_pass(m == -INFINITY ? 0.f : m);
+            store_p();
+            l += (rs01.x + rs01.y) + (rs23.x + rs23.y);
             if (ntiles > 0 && any) {
                 // this warpgroup's O must be complete before it is rescaled
                 // (PV(t) is issued only after p_full below).  Waiting only when
