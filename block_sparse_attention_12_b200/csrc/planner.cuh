@@ -21,13 +21,16 @@ namespace abattn {
 
 constexpr int PL_THREADS = 512;
 constexpr int PL_WARPS = PL_THREADS / 32;
-// Capping candidates: blocks left uncapped by the first round whose score is
-// within a factor PL_CAND_ALPHA of that round's threshold.  The later rounds
-// test only these while lambda stays below PL_CAND_ALPHA times its first value
-// (so no other block can reach the threshold); otherwise, or when more than
-// PL_CAND blocks qualify, every round scans the whole row.
+// Capping candidates: blocks whose score is within a factor PL_CAND_ALPHA of
+// the first threshold 1 / lambda_0, listed while the row loads (or, for rows
+// that sum to less than 0.9, by a first round over the whole row).  The
+// rounds test only these while lambda stays below PL_CAND_ALPHA lambda_0 (so
+// no other block can reach the threshold); otherwise, or when a warp lists
+// more than PL_CAND_W blocks, every round scans the whole row.  On the
+// workloads' score rows lambda ends 6 to 22 times above lambda_0.
 constexpr int PL_CAND = 2048;
-constexpr double PL_CAND_ALPHA = 64.0;
+constexpr int PL_CAND_W = PL_CAND / (PL_THREADS / 32);  // per-warp region of the list
+constexpr double PL_CAND_ALPHA = 32.0;
 
 enum PlanMode : int { kPlanSip = 0, kPlanTopk = 1, kPlanFromPi = 2 };
 
@@ -81,6 +84,18 @@ __device__ __forceinline__ void load8(const float *vals, int j0, int end, float 
     }
 }
 
+// vals[j0 .. j0+7] = r (only the entries below `end`).
+__device__ __forceinline__ void store8(float *vals, int j0, int end, const float (&r)[8]) {
+    if (j0 + 8 <= end) {
+        *reinterpret_cast<float4 *>(vals + j0) = make_float4(r[0], r[1], r[2], r[3]);
+        *reinterpret_cast<float4 *>(vals + j0 + 4) = make_float4(r[4], r[5], r[6], r[7]);
+    } else {
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            if (j0 + u < end) vals[j0 + u] = r[u];
+    }
+}
+
 struct PlanScratch {
     int iwarp[PL_WARPS];
     double dwarp[PL_WARPS];
@@ -89,8 +104,8 @@ struct PlanScratch {
     int bcast[4];
     double dbcast;
     int hist[256];
-    int ncand;
-    uint16_t cand[PL_CAND];
+    int wcand[PL_WARPS];      // candidates listed by each warp (may exceed PL_CAND_W)
+    uint16_t cand[PL_CAND];   // warp w's candidates at [w * PL_CAND_W, ...)
 };
 
 // Block-wide sums of one int and one double in a single exchange.
@@ -160,10 +175,17 @@ __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
     const int nbytes = ((n + 31) / 32) * 4;
 
     // load (8 independent loads in flight per thread); SIP also counts
-    // positive scores and sums them
+    // positive scores, sums them and lists the capping candidates: the
+    // blocks with s >= 0.9 / (PL_CAND_ALPHA Bblk).  When the row sums to at
+    // least 0.9 (scores sum to 1) that bound is below 1 / (PL_CAND_ALPHA
+    // lambda_0), so the list holds every block that a lambda up to
+    // PL_CAND_ALPHA lambda_0 can cap.
     int npos_l = 0;
     double sum_l = 0.0;
-    for (int j0 = tid; j0 < n; j0 += 8 * PL_THREADS) {
+    const float cand_thr = MODE == kPlanSip ? float(0.9 / (PL_CAND_ALPHA * Bblk)) * (1.f - 1e-5f) : 0.f;
+    int ncw = 0;  // candidates this warp has listed (warp-uniform)
+    uint16_t *wcand_list = sc.cand + wid * PL_CAND_W;
+    for (int j0 = tid; j0 - lane < n; j0 += 8 * PL_THREADS) {
         float v[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
@@ -180,15 +202,29 @@ __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
                     sum_l += double(v[u]);
                 }
             }
+            if (MODE == kPlanSip) {
+                // appended to this warp's region of the list, no atomics
+                const bool c = j < n && v[u] >= cand_thr;
+                const uint32_t cm = __ballot_sync(0xffffffffu, c);
+                const int at = ncw + __popc(cm & ((1u << lane) - 1u));
+                if (c && at < PL_CAND_W) wcand_list[at] = uint16_t(j);
+                ncw += __popc(cm);
+            }
         }
     }
     for (int i = tid; i < nbytes; i += PL_THREADS) flags[i] = 0;
+    if (MODE == kPlanSip && lane == 0) sc.wcand[wid] = ncw;
 
     // this warp's segment; lane works on blocks j0 .. j0+7 of each 256-block step
     const int seg = ((n + PL_WARPS * 256 - 1) / (PL_WARPS * 256)) * 256;
     const int w0 = wid * seg;
     const int w1 = w0 + seg < n ? w0 + seg : n;
 
+    // SIP: after the capping rounds vals still holds the scores; the sampling
+    // pass takes pi = 1 for capped blocks (their flag bits) and
+    // fp32(lambda s) for the others
+    bool pi_from_s = false;
+    double lam_final = 0.0;
     if (MODE == kPlanSip) {
         const int npos = block_sum<int>(npos_l, sc.iwarp, &sc.bcast[0]);  // (also orders the loads)
         if (Bblk >= double(npos)) {
@@ -201,8 +237,17 @@ __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
             // walk (conflict-free shared loads); the capped flags of 32
             // consecutive blocks form one word, rebuilt by ballot.
             uint32_t *fw = reinterpret_cast<uint32_t *>(flags);
-            if (tid == 0) sc.ncand = 0;
-            double rest = block_sum<double>(sum_l, sc.dwarp, &sc.dbcast);  // (also publishes ncand = 0)
+            double rest = block_sum<double>(sum_l, sc.dwarp, &sc.dbcast);  // (also publishes wcand)
+            auto cand_fit = [&]() {
+                bool fit = true;
+#pragma unroll
+                for (int w = 0; w < PL_WARPS; ++w) fit &= sc.wcand[w] <= PL_CAND_W;
+                return fit;
+            };
+            // the load pass's list serves when it is complete and the row sums
+            // to at least 0.9; otherwise the first round scans the whole row
+            // and lists the candidates itself
+            const bool pre_ok = rest >= 0.9 && cand_fit();
             int ncap = 0;
             double lam = Bblk / rest;
             const double lam_lim = PL_CAND_ALPHA * lam;
@@ -212,6 +257,7 @@ __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
                 const float cand_near = float(lam_lim) * (1.f + 1e-5f);
                 int added_l = 0;
                 double capped_l = 0.0;
+                int nc = 0;  // candidates this warp has listed (warp-uniform)
                 // four words (128 blocks) per step: four independent chains
                 for (int j128 = w0; j128 < w1; j128 += 128) {
                     uint32_t word[4];
@@ -237,24 +283,44 @@ __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
                         if (collect) {
                             const bool c = open && !cap_now && sv[q] * cand_near >= 1.f;
                             const uint32_t cm = __ballot_sync(0xffffffffu, c);
-                            if (cm != 0u) {
-                                int base = 0;
-                                if (lane == 0) base = atomicAdd(&sc.ncand, __popc(cm));
-                                base = __shfl_sync(0xffffffffu, base, 0);
-                                const int at = base + __popc(cm & ((1u << lane) - 1u));
-                                if (c && at < PL_CAND) sc.cand[at] = uint16_t(j);
-                            }
+                            const int at = nc + __popc(cm & ((1u << lane) - 1u));
+                            if (c && at < PL_CAND_W) wcand_list[at] = uint16_t(j);
+                            nc += __popc(cm);
                         }
+                    }
+                }
+                if (collect && lane == 0) sc.wcand[wid] = nc;
+                block_sum2(added_l, capped_l, sc, added, capped);
+            };
+            // a round over the candidates only, each warp over its own list
+            auto cand_round = [&](int &added, double &capped) {
+                const float near = float(lam) * (1.f + 1e-5f);
+                int added_l = 0;
+                double capped_l = 0.0;
+                const int cw = sc.wcand[wid];
+                for (int i = lane; i < cw; i += 32) {
+                    const int j = wcand_list[i];
+                    const float sj = vals[j];
+                    const uint32_t bit = 1u << (j & 31);
+                    if (!(fw[j >> 5] & bit) && sj * near >= 1.f && lam * double(sj) >= 1.0) {
+                        atomicOr(&fw[j >> 5], bit);
+                        ++added_l;
+                        capped_l += double(sj);
                     }
                 }
                 block_sum2(added_l, capped_l, sc, added, capped);
             };
             int added;
             double capped;
-            full_round(true, added, capped);
-            const bool cand_ok = sc.ncand <= PL_CAND;  // read after block_sum2's barriers
-            const int ncand = sc.ncand;
-            bool scan_all = !cand_ok;
+            bool scan_all;
+            if (pre_ok) {
+                scan_all = false;
+                cand_round(added, capped);
+            } else {
+                __syncthreads();  // every thread has read wcand before the first round relists
+                full_round(true, added, capped);
+                scan_all = !cand_fit();  // wcand read after block_sum2's barriers
+            }
             while (added != 0) {
                 rest -= capped;
                 ncap += added;
@@ -263,37 +329,14 @@ __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
                 if (scan_all) {
                     full_round(false, added, capped);
                 } else {
-                    // a round over the candidates only
-                    const float near = float(lam) * (1.f + 1e-5f);
-                    int added_l = 0;
-                    double capped_l = 0.0;
-                    for (int i = tid; i < ncand; i += PL_THREADS) {
-                        const int j = sc.cand[i];
-                        const float sj = vals[j];
-                        const uint32_t bit = 1u << (j & 31);
-                        if (!(fw[j >> 5] & bit) && sj * near >= 1.f && lam * double(sj) >= 1.0) {
-                            atomicOr(&fw[j >> 5], bit);
-                            ++added_l;
-                            capped_l += double(sj);
-                        }
-                    }
-                    block_sum2(added_l, capped_l, sc, added, capped);
+                    cand_round(added, capped);
                 }
             }
-            // pi into shared memory (lane-strided, conflict-free); the capped
-            // flags are cleared again for the sampling pass
-            for (int j32 = w0; j32 < w1; j32 += 32) {
-                const int j = j32 + lane;
-                const uint32_t word = fw[j32 >> 5];
-                if (j < w1) vals[j] = ((word >> lane) & 1u) ? 1.f : __double2float_rn(lam * double(vals[j]));
-                __syncwarp();
-                if (lane == 0) fw[j32 >> 5] = 0u;
-            }
+            pi_from_s = true;
+            lam_final = lam;
         }
     }
     __syncthreads();
-    if (MODE == kPlanSip && pi_out != nullptr)
-        for (int j = tid; j < n; j += PL_THREADS) pi_out[row * nkvb + j] = vals[j];
 
     // top-k threshold: radix select on the fp32 bit patterns of the
     // non-negative scores, 8 bits per pass, most significant first
@@ -346,6 +389,14 @@ __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
         } else {
             float pv[8];
             load8(vals, j0, w1, pv);
+            if (pi_from_s) {
+                // this lane's 8 blocks: pi from the capped bits and lambda
+                const uint32_t cb = flags[j0 >> 3];
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    pv[u] = ((cb >> u) & 1u) ? 1.f : __double2float_rn(lam_final * double(pv[u]));
+                store8(vals, j0, w1, pv);
+            }
             float u8[8];
             row_uniforms8(seed, b, h, qb, j0 >> 3, u8);
 #pragma unroll
@@ -362,6 +413,8 @@ __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
         sc.wcount2[wid] = neq_w;
     }
     __syncthreads();
+    if (MODE == kPlanSip && pi_out != nullptr)
+        for (int j = tid; j < n; j += PL_THREADS) pi_out[row * nkvb + j] = vals[j];
     int pos = 0, eq_rank = 0, total = 0, eq_total = 0;
     for (int w = 0; w < PL_WARPS; ++w) {
         if (w < wid) {

@@ -210,16 +210,23 @@ def test_waterfill_pi_parity(tiny):
 
 def _fallback_rows(n, rng):
     """Score rows for the water-fill's fallback paths (n = 4096 blocks, 8%
-    budget): (a) lambda grows past 64 times its first value, so the rounds
-    after the first scan the whole row (and cap 100 more blocks); (b) more
-    than 2048 blocks qualify as candidates, so the list overflows and a full
-    round caps 200 more; (c) an ordinary heavy-tailed row (candidate rounds)."""
+    budget; the kernel lists as capping candidates the blocks within a factor
+    32 of the first threshold): (a) lambda grows past 32 times its first
+    value, so the rounds after the first scan the whole row (and cap 100 more
+    blocks); (b) more than 2048 blocks qualify as candidates, so the list
+    overflows and the later rounds scan the row; (c) an ordinary heavy-tailed
+    row;
+    (d) the same row normalised to sum 1, as scores are, whose candidates are
+    listed while the row loads; (e) row (d) times 1/4, whose sum is below 1/2,
+    so the first round scans the row instead."""
     a = np.concatenate([np.full(60, 1e6), np.full(100, 40.0), np.full(n - 160, 1.0)])
-    b = np.concatenate([np.full(60, 2000.0), np.full(200, 500.0), np.full(2100, 12.0), np.full(n - 2360, 0.1)])
+    b = np.concatenate([np.full(60, 2000.0), np.full(200, 500.0), np.full(2100, 40.0), np.full(n - 2360, 0.1)])
     c = np.exp(rng.standard_normal(n) * 2.0)
+    d = np.exp(rng.standard_normal(n) * 3.0)
+    d = d / d.sum()
     for r in (a, b):
         rng.shuffle(r)
-    return [a, b, c]
+    return [a, b, c, d, d * 0.25]
 
 
 def test_waterfill_fallback_paths():
@@ -232,17 +239,18 @@ def test_waterfill_fallback_paths():
     # the rows take the paths they are built for
     lam0 = [Bblk / r.sum() for r in rows]
     pis = [oracle.waterfill(r, Bblk) for r in rows]
-    assert pis[0][1] / lam0[0] > 64
-    assert ((rows[1] * 64 * lam0[1] >= 1) & (rows[1] * lam0[1] < 1)).sum() > 2048
-    assert (pis[0][0] >= 1).sum() == 160 and (pis[1][0] >= 1).sum() == 260
+    assert pis[0][1] / lam0[0] > 32
+    assert ((rows[1] * 32 * lam0[1] >= 1) & (rows[1] * lam0[1] < 1)).sum() > 2048
+    assert (pis[0][0] >= 1).sum() == 160 and (pis[1][0] >= 1).sum() == 60
     S = np.tile(rows[2], (N // 128, 1))
     S[:2] = rows[0], rows[1]
+    S[3:5] = rows[3], rows[4]
     S32 = torch.from_numpy(S.astype(np.float32)).reshape(B, H, N // 128, n)
     pg, pig = abi.plan_from_scores(S32.cuda(), (B, H, N, d), cfg, want_pi=True)
     abi.check()
     pig = pig.cpu().numpy()[0, 0]
     counts, idx, ps = (t.cpu().numpy()[0, 0] for t in (pg.counts, pg.idx, pg.pi_sel))
-    for qb in (0, 1, 2, N // 128 - 1):
+    for qb in (0, 1, 2, 3, 4, N // 128 - 1):
         po, _, _ = oracle.waterfill(S32[0, 0, qb].double().numpy(), Bblk)
         assert np.max(np.abs(pig[qb] - po) / np.maximum(po, 1e-30)) <= 1e-5, qb
         idx_o, ps_o, n_o = oracle.sample(pig[qb], cfg.seed, 0, 0, qb, pg.cap)
