@@ -99,6 +99,8 @@ __device__ __forceinline__ void store8(float *vals, int j0, int end, const float
 struct PlanScratch {
     int iwarp[PL_WARPS];
     double dwarp[PL_WARPS];
+    int iwarp2[2][PL_WARPS];
+    double dwarp2[2][PL_WARPS];
     int wcount[PL_WARPS];   // per-warp selected (or tie) counts
     int wcount2[PL_WARPS];
     int bcast[4];
@@ -108,26 +110,28 @@ struct PlanScratch {
     uint16_t cand[PL_CAND];   // warp w's candidates at [w * PL_CAND_W, ...)
 };
 
-// Block-wide sums of one int and one double in a single exchange.
-__device__ __forceinline__ void block_sum2(int vi, double vd, PlanScratch &sc, int &si, double &sd) {
+// Block-wide sums of one int and one double in a single exchange, with one
+// barrier: the warp partials alternate between two buffers (flipped by
+// `parity`), so a round's writes never meet the previous round's reads.
+__device__ __forceinline__ void block_sum2(int vi, double vd, PlanScratch &sc, int &parity, int &si, double &sd) {
     vi = warp_sum(vi);
     vd = warp_sum(vd);
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     if (lane == 0) {
-        sc.iwarp[wid] = vi;
-        sc.dwarp[wid] = vd;
+        sc.iwarp2[parity][wid] = vi;
+        sc.dwarp2[parity][wid] = vd;
     }
     __syncthreads();
     int ti = 0;
     double td = 0.0;
 #pragma unroll
     for (int w = 0; w < PL_WARPS; ++w) {
-        ti += sc.iwarp[w];
-        td += sc.dwarp[w];
+        ti += sc.iwarp2[parity][w];
+        td += sc.dwarp2[parity][w];
     }
     si = ti;
     sd = td;
-    __syncthreads();
+    parity ^= 1;
 }
 
 // Block-wide sum; every thread gets the result.
@@ -249,6 +253,7 @@ __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
             // and lists the candidates itself
             const bool pre_ok = rest >= 0.9 && cand_fit();
             int ncap = 0;
+            int rpar = 0;  // buffer parity of block_sum2
             double lam = Bblk / rest;
             const double lam_lim = PL_CAND_ALPHA * lam;
             // one round over the whole row; the first one also collects the candidates
@@ -290,7 +295,7 @@ __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
                     }
                 }
                 if (collect && lane == 0) sc.wcand[wid] = nc;
-                block_sum2(added_l, capped_l, sc, added, capped);
+                block_sum2(added_l, capped_l, sc, rpar, added, capped);
             };
             // a round over the candidates only, each warp over its own list
             auto cand_round = [&](int &added, double &capped) {
@@ -308,7 +313,7 @@ __global__ void __launch_bounds__(PL_THREADS) plan_kernel(
                         capped_l += double(sj);
                     }
                 }
-                block_sum2(added_l, capped_l, sc, added, capped);
+                block_sum2(added_l, capped_l, sc, rpar, added, capped);
             };
             int added;
             double capped;
