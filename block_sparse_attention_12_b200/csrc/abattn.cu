@@ -170,15 +170,18 @@ template <int D>
 int launch_kmeans_t(const void *Q, const abattn_dims *d, const abattn_params *p, float *C, float *w,
                     int32_t *labels, __nv_bfloat16 *Chi, __nv_bfloat16 *Clo, cudaStream_t st) {
     const int64_t nqb = cdiv(d->N, 128), rows = d->B * d->H * nqb;
-    constexpr size_t smem = kmeans_smem_bytes<D>();
+    constexpr int smem = KmLayout::ALLOC;
     static bool attr = false;
     if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(kmeans_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        cudaError_t e = cudaFuncSetAttribute(kmeans_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return cuda_status(e);
         attr = true;
     }
-    kmeans_kernel<D><<<unsigned(rows), KM_THREADS, smem, st>>>(
-        static_cast<const __nv_bfloat16 *>(Q), d->N, nqb, p->n_clusters, p->kmeans_iters, C, w, labels, Chi, Clo);
+    CUtensorMap mQ;
+    int rc = make_map(&mQ, Q, d, 128);
+    if (rc) return rc;
+    kmeans_kernel<D><<<unsigned(rows), KM_THREADS, smem, st>>>(mQ, d->N, nqb, p->n_clusters, p->kmeans_iters, C, w,
+                                                               labels, Chi, Clo);
     return launch_status();
 }
 

@@ -88,83 +88,124 @@ __global__ void split_rows_kernel(const float *__restrict__ src, int64_t nblk, i
 }
 
 // ---------------------------------------------------------------- k-means
-// One CTA (128 threads) per q-block.  The block's queries sit in shared
-// memory transposed and in their own bf16 precision, Qs[k][i] (row stride
-// 130 bf16: conflict-free column and row walks); centroids fp32,
-// interleaved, Cs[k][8].
-//   assignment: thread i scores its query against all 8 centroids as
-//               |c|^2 - 2 q.c (the same argmin as |q - c|^2; |q|^2 is
-//               common), ties to the lower index;
-//   update:     a stable counting sort of the labels (warp ballots) gives
-//               each cluster's members in ascending query order; thread k
-//               sums column k over each cluster's members.
+// One CTA (128 threads, one warpgroup) per q-block; both Lloyd steps run on
+// the tensor cores, with the block's queries staged once by TMA in the
+// 128-byte-swizzled K-major layout:
+//   assignment: D_a[query][c] = q . c for 16 centroid slots (8 used) as
+//               Q [128 x d] times (C_hi + C_lo)^T, two bf16 MMA groups into
+//               one fp32 TMEM accumulator (the queries are exactly bf16, the
+//               fp32 centroids split into a bf16 pair hi + lo); thread i
+//               (TMEM lane i) then takes argmin_c |c|^2 - 2 q.c (the same
+//               argmin as |q - c|^2), ties to the lower index;
+//   update:     D_u[k][c] = sum of dimension k over cluster c's members as
+//               Q^T [d x 128] times a one-hot [128 x 16] assignment matrix;
+//               the same shared-memory tile of Q is read as an MN-major
+//               operand; thread k divides by the member counts (ballots).
+// Products are exact (bf16 x bf16, or x 0/1) and accumulate in fp32.  An
+// empty cluster keeps its centroid; a fixed point (no label moved) ends the
+// iterations early with the same result.  For d = 64 the tile's second
+// 64-column half is zero, so the update still has M = 128 rows.
 constexpr int KM_THREADS = 128;
-constexpr int KM_QS = 130;  // bf16 elements per Qs row (65 words: odd stride)
 
-template <int D>
-constexpr size_t kmeans_smem_bytes() {
-    return sizeof(__nv_bfloat16) * size_t(D) * KM_QS + sizeof(float) * (size_t(D) * 8 + 8 + 4 * 8) +
-           sizeof(int) * (128 + 128 + 8 + 9 + 4 * 8);
+struct KmLayout {
+    static constexpr int Q_OFF = 0;          // [2 halves][128 rows][128 B]
+    static constexpr int CHI_OFF = 32768;    // [2 halves][16 rows][128 B]
+    static constexpr int CLO_OFF = 36864;
+    static constexpr int OH_OFF = 40960;     // one-hot, [2 query halves][16 rows][128 B]
+    static constexpr int CS_OFF = 45056;     // fp32 centroids [8][128]
+    static constexpr int CN_OFF = CS_OFF + 8 * 128 * 4;  // |c|^2 [8], partials [4][8]
+    static constexpr int INT_OFF = CN_OFF + 40 * 4;      // lab[128], cnt[8], wcnt[4][8]
+    static constexpr int BAR_OFF = INT_OFF + (128 + 8 + 32) * 4;  // q_bar, mma_bar
+    static constexpr int MISC_OFF = BAR_OFF + 16;         // tmem slot
+    static constexpr int BYTES = MISC_OFF + 16;
+    static constexpr int ALLOC = BYTES + 1024;
+};
+
+// Byte offset of element (r, k) in a 128-byte-swizzled K-major tile whose
+// 64-column halves are `hs` bytes apart (rows of 128 bytes).
+__device__ __forceinline__ uint32_t sw128_off(int r, int k, uint32_t hs) {
+    const int cc = k & 63;
+    return uint32_t(k >> 6) * hs + uint32_t(r) * 128u + (uint32_t(((cc >> 3) ^ (r & 7))) << 4) + uint32_t(cc & 7) * 2u;
 }
 
 template <int D>
 __global__ void __launch_bounds__(KM_THREADS) kmeans_kernel(
-    const __nv_bfloat16 *__restrict__ Q, int64_t N, int64_t nqb, int nc, int iters,
+    const __grid_constant__ CUtensorMap tmQ, int64_t N, int64_t nqb, int nc, int iters,
     float *__restrict__ Cout, float *__restrict__ wout, int32_t *__restrict__ labels_out,
     __nv_bfloat16 *__restrict__ Chi, __nv_bfloat16 *__restrict__ Clo) {
-    extern __shared__ float km_smem[];
-    __nv_bfloat16 *Qs = reinterpret_cast<__nv_bfloat16 *>(km_smem);               // [D][KM_QS]
-    float *Cs = km_smem + (D * KM_QS) / 2;                                         // [D][8]
-    float *cn = Cs + D * 8;                       // [8]     |c|^2
-    float *cn_part = cn + 8;                      // [4][8]  per-warp partial |c|^2
-    int *lab = reinterpret_cast<int *>(cn_part + 32);  // [128]
-    int *order = lab + 128;                        // [128]   queries sorted by cluster
-    int *cnt_s = order + 128;                      // [8]
-    int *start = cnt_s + 8;                        // [9]
-    int *wcnt = start + 9;                         // [4][8]  per-warp cluster counts
+    using L = KmLayout;
+    extern __shared__ uint8_t km_smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(km_smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sQ = smem + L::Q_OFF;
+    uint8_t *sChi = smem + L::CHI_OFF, *sClo = smem + L::CLO_OFF, *sOH = smem + L::OH_OFF;
+    float *Cs = reinterpret_cast<float *>(smem + L::CS_OFF);   // [8][D]
+    float *cn = reinterpret_cast<float *>(smem + L::CN_OFF);   // [8]
+    float *cn_part = cn + 8;                                    // [4][8]
+    int *lab = reinterpret_cast<int *>(smem + L::INT_OFF);     // [128]
+    int *cnt_s = lab + 128;                                     // [8]
+    int *wcnt = cnt_s + 8;                                      // [4][8]
+    uint64_t *q_bar = reinterpret_cast<uint64_t *>(smem + L::BAR_OFF);
+    uint64_t *mma_bar = q_bar + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::MISC_OFF);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::MISC_OFF + 4);
 
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int64_t row = blockIdx.x;
     const int64_t bh = row / nqb, qb = row % nqb;
-    const int64_t q0 = qb * 128;
+    const int q0 = int(qb * 128);
     const int M = int(N - q0 < 128 ? N - q0 : 128);
 
-    // load (all 16-byte loads in flight first) + transpose
-    constexpr int G = D / 8;
-    constexpr int PER = (128 * G) / KM_THREADS;  // 16-byte chunks per thread
-    const __nv_bfloat16 *src = Q + (bh * N + q0) * D;
+    if (wid == 0) {
+        tmem_alloc(tmem_slot, 32);  // D_a: columns [0, 16), D_u: [16, 32)
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        mbar_init(q_bar, 1);
+        mbar_init(mma_bar, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    // zero the centroid and one-hot operands (their unused rows stay zero)
+    // and, for d = 64, the tile's second half
     {
-        uint4 v[PER];
-#pragma unroll
-        for (int u = 0; u < PER; ++u) {
-            const int e = tid + u * KM_THREADS, i = e / G, c8 = e % G;
-            v[u] = i < M ? __ldg(reinterpret_cast<const uint4 *>(src + size_t(i) * D + c8 * 8)) : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int u = 0; u < PER; ++u) {
-            const int e = tid + u * KM_THREADS, i = e / G, c8 = e % G;
-            const __nv_bfloat16 *hv = reinterpret_cast<const __nv_bfloat16 *>(&v[u]);
-#pragma unroll
-            for (int x = 0; x < 8; ++x) Qs[(c8 * 8 + x) * KM_QS + i] = hv[x];
+        uint4 *z = reinterpret_cast<uint4 *>(smem + L::CHI_OFF);
+        for (int e = tid; e < (3 * 4096) / 16; e += KM_THREADS) z[e] = make_uint4(0, 0, 0, 0);
+        if (D == 64) {
+            uint4 *zq = reinterpret_cast<uint4 *>(sQ + 16384);
+            for (int e = tid; e < 16384 / 16; e += KM_THREADS) zq[e] = make_uint4(0, 0, 0, 0);
         }
     }
+    tc_fence_before();
     __syncthreads();
-    // init: centroid c = query floor(c*M/nc); unused centroid slots are zero
-    for (int e = tid; e < D * 8; e += KM_THREADS) {
-        const int k = e / 8, c = e % 8;
-        Cs[e] = c < nc ? __bfloat162float(Qs[k * KM_QS + (c * M) / nc]) : 0.f;
-    }
-    if (tid < 8) cnt_s[tid] = 0;
-    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t t_lane = tmem + (uint32_t(wid * 32) << 16);
 
-    auto centroid_norms = [&]() {
-        float part[8];
+    bool ok = true;
+    if (tid == 0) {
+        mbar_arrive_expect_tx(q_bar, 128 * D * 2);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) part[c] = 0.f;
-        for (int k = tid; k < D; k += KM_THREADS) {
-#pragma unroll
-            for (int c = 0; c < 8; ++c) part[c] = fmaf(Cs[k * 8 + c], Cs[k * 8 + c], part[c]);
-        }
+        for (int h = 0; h < D / 64; ++h) tma_load_3d(sQ + h * 16384, &tmQ, q_bar, h * 64, q0, int(bh));
+    }
+    ok = mbar_wait(q_bar, 0, abort_flag);
+    ok = __syncthreads_and(ok) != 0;
+
+    auto qval = [&](int r, int k) {
+        return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sQ + sw128_off(r, k, 16384)));
+    };
+    // centroid c of dimension k (thread k) into Cs and the bf16 hi/lo operand
+    // tiles; returns its square for |c|^2
+    auto set_centroid = [&](int c, int k, float v) {
+        Cs[c * D + k] = v;
+        __nv_bfloat16 hi, lo;
+        split_bf16(v, hi, lo);
+        const uint32_t o = sw128_off(c, k, 2048);
+        *reinterpret_cast<__nv_bfloat16 *>(sChi + o) = hi;
+        *reinterpret_cast<__nv_bfloat16 *>(sClo + o) = lo;
+        return v * v;
+    };
+    // |c|^2 from each thread's dimension: warp sums, then across the warps
+    auto centroid_norms = [&](const float (&part)[8]) {
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
             const float v = warp_sum(part[c]);
@@ -172,99 +213,126 @@ __global__ void __launch_bounds__(KM_THREADS) kmeans_kernel(
         }
         __syncthreads();
         if (tid < 8) cn[tid] = (cn_part[tid] + cn_part[8 + tid]) + (cn_part[16 + tid] + cn_part[24 + tid]);
-        __syncthreads();
     };
-    if (iters > 0) centroid_norms();
 
-    for (int it = 0; it < iters; ++it) {
-        // assignment
-        int best = 0;
-        if (tid < M) {
-            float a[8];
+    // init: centroid c = query floor(c*M/nc); unused centroid slots are zero
+    {
+        float part[8];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) a[c] = 0.f;
-#pragma unroll 4
-            for (int k = 0; k < D; ++k) {
-                const float q = __bfloat162float(Qs[k * KM_QS + tid]);
-                const float4 c0 = *reinterpret_cast<const float4 *>(Cs + k * 8);
-                const float4 c1 = *reinterpret_cast<const float4 *>(Cs + k * 8 + 4);
-                a[0] = fmaf(q, c0.x, a[0]);
-                a[1] = fmaf(q, c0.y, a[1]);
-                a[2] = fmaf(q, c0.z, a[2]);
-                a[3] = fmaf(q, c0.w, a[3]);
-                a[4] = fmaf(q, c1.x, a[4]);
-                a[5] = fmaf(q, c1.y, a[5]);
-                a[6] = fmaf(q, c1.z, a[6]);
-                a[7] = fmaf(q, c1.w, a[7]);
+        for (int c = 0; c < 8; ++c) {
+            const float v = (tid < D && c < nc) ? qval((c * M) / nc, tid < D ? tid : 0) : 0.f;
+            part[c] = tid < D ? set_centroid(c, tid, v) : 0.f;
+        }
+        fence_proxy_async_smem();
+        centroid_norms(part);
+    }
+    if (tid < 8) cnt_s[tid] = 0;
+
+    constexpr uint32_t idesc_a = make_idesc_bf16(128, 16, 0, 0);  // Q . C^T
+    constexpr uint32_t idesc_u = make_idesc_bf16(128, 16, 1, 0);  // Q^T . onehot, A MN-major
+    uint32_t phase = 0;
+    for (int it = 0; ok && it < iters; ++it) {
+        __syncthreads();  // centroid operands, |c|^2 and the last one-hot reads are done
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t q_lo = sdesc_lo(smem_u32(sQ), 16);
+            const uint32_t hi_lo = sdesc_lo(smem_u32(sChi), 16), lo_lo = sdesc_lo(smem_u32(sClo), 16);
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k) {
+                const uint32_t qo = ((k >> 2) * 16384 + (k & 3) * 32) >> 4, co = ((k >> 2) * 2048 + (k & 3) * 32) >> 4;
+                umma_ss_lo(tmem, q_lo + qo, hi_lo + co, idesc_a, k > 0 ? 1u : 0u);
             }
-            float bd = fmaf(-2.f, a[0], cn[0]);
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k) {
+                const uint32_t qo = ((k >> 2) * 16384 + (k & 3) * 32) >> 4, co = ((k >> 2) * 2048 + (k & 3) * 32) >> 4;
+                umma_ss_lo(tmem, q_lo + qo, lo_lo + co, idesc_a, 1u);
+            }
+            umma_commit(mma_bar);
+        }
+        ok = mbar_wait(mma_bar, phase, abort_flag);
+        phase ^= 1;
+        tc_fence_after();
+        uint32_t a16[16];
+        tmem_ld16(t_lane, a16);
+        tmem_wait_ld();
+        int best = 0;
+        {
+            float bd = fmaf(-2.f, __uint_as_float(a16[0]), cn[0]);
 #pragma unroll
             for (int c = 1; c < 8; ++c) {
-                const float v = fmaf(-2.f, a[c], cn[c]);
+                const float v = fmaf(-2.f, __uint_as_float(a16[c]), cn[c]);
                 if (c < nc && v < bd) { bd = v; best = c; }
             }
         }
         // a fixed point (no label changed) repeats itself in every remaining
         // iteration: stop, the result is the same as running them all
         const bool moved = tid < M && (it == 0 || lab[tid] != best);
-        if (it > 0 && !__syncthreads_or(moved)) break;
+        const int flags = __syncthreads_or((moved ? 1 : 0) | (ok ? 0 : 2));
+        if (flags & 2) { ok = false; break; }
+        if (it > 0 && !(flags & 1)) break;
         if (tid < M) lab[tid] = best;
-        // stable counting sort of the labels
-        unsigned my_rank = 0;
+        // member counts and the one-hot operand (column tid)
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
             const unsigned m = __ballot_sync(0xffffffffu, tid < M && best == c);
-            if (best == c) my_rank = __popc(m & ((1u << lane) - 1u));
             if (lane == 0) wcnt[wid * 8 + c] = __popc(m);
+            const __nv_bfloat16 one = __float2bfloat16(tid < M && best == c ? 1.f : 0.f);
+            *reinterpret_cast<__nv_bfloat16 *>(sOH + sw128_off(c, tid, 2048)) = one;
         }
+        fence_proxy_async_smem();
+        tc_fence_before();
         __syncthreads();
+        if (tid < 8) cnt_s[tid] = wcnt[tid] + wcnt[8 + tid] + wcnt[16 + tid] + wcnt[24 + tid];
         if (tid == 0) {
-            int acc = 0;
-            for (int c = 0; c < 8; ++c) {
-                start[c] = acc;
-                const int n = wcnt[c] + wcnt[8 + c] + wcnt[16 + c] + wcnt[24 + c];
-                cnt_s[c] = n;
-                acc += n;
-            }
-            start[8] = acc;
-        }
-        __syncthreads();
-        if (tid < M) {
-            int pos = start[best] + int(my_rank);
-            for (int w = 0; w < wid; ++w) pos += wcnt[w * 8 + best];
-            order[pos] = tid;
-        }
-        __syncthreads();
-        // update: thread k sums column k over each cluster's members (ascending order)
-        for (int k = tid; k < D; k += KM_THREADS) {
+            tc_fence_after();
+            const uint32_t qt_lo = sdesc_lo(smem_u32(sQ), 16384), oh_lo = sdesc_lo(smem_u32(sOH), 16);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
+            for (int k = 0; k < 8; ++k) {
+                const uint32_t oo = ((k >> 2) * 2048 + (k & 3) * 32) >> 4;
+                umma_ss_lo(tmem + 16, qt_lo + k * (2048 >> 4), oh_lo + oo, idesc_u, k > 0 ? 1u : 0u);
+            }
+            umma_commit(mma_bar);
+        }
+        ok = mbar_wait(mma_bar, phase, abort_flag);
+        phase ^= 1;
+        tc_fence_after();
+        uint32_t s16[16];
+        tmem_ld16(t_lane + 16, s16);
+        tmem_wait_ld();
+        ok = __syncthreads_and(ok) != 0;  // (also publishes cnt_s)
+        if (!ok) break;
+        float part[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            part[c] = 0.f;
+            if (tid < D) {
                 const int n = cnt_s[c];
-                if (c < nc && n > 0) {
-                    float acc = 0.f;
-                    for (int p = start[c]; p < start[c + 1]; ++p) acc += __bfloat162float(Qs[k * KM_QS + order[p]]);
-                    Cs[k * 8 + c] = acc / float(n);
-                }
+                const float v = (c < nc && n > 0) ? __uint_as_float(s16[c]) / float(n) : Cs[c * D + tid];
+                part[c] = set_centroid(c, tid, v);
             }
         }
-        __syncthreads();
-        if (it + 1 < iters) centroid_norms();
+        fence_proxy_async_smem();
+        centroid_norms(part);
     }
+    __syncthreads();
 
-    const int64_t r = row;
     if (Cout != nullptr)
-        for (int e = tid; e < nc * D; e += KM_THREADS) {
-            const int c = e / D, k = e % D;
-            Cout[(r * nc + c) * D + k] = Cs[k * 8 + c];
-        }
+        for (int e = tid; e < nc * D; e += KM_THREADS) Cout[row * nc * D + e] = Cs[e];
     if (Chi != nullptr)  // [rows][8][D], clusters past nc zero
         for (int e = tid; e < 8 * D; e += KM_THREADS) {
-            const int c = e / D, k = e % D;
-            split_bf16(c < nc ? Cs[k * 8 + c] : 0.f, Chi[(r * 8 + c) * D + k], Clo[(r * 8 + c) * D + k]);
+            const int c = e / D;
+            split_bf16(c < nc ? Cs[e] : 0.f, Chi[row * 8 * D + e], Clo[row * 8 * D + e]);
         }
-    if (tid < nc) wout[r * nc + tid] = iters > 0 ? float(cnt_s[tid]) / float(M) : 1.f / float(nc);
-    if (labels_out != nullptr && tid < 128)
-        labels_out[r * 128 + tid] = (iters > 0 && tid < M) ? lab[tid] : -1;
+    if (tid < nc) wout[row * nc + tid] = iters > 0 ? float(cnt_s[tid]) / float(M) : 1.f / float(nc);
+    if (labels_out != nullptr)
+        labels_out[row * 128 + tid] = (iters > 0 && tid < M) ? lab[tid] : -1;
+
+    tc_fence_before();
+    __syncthreads();
+    if (wid == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 32);
+    }
 }
 
 // ---------------------------------------------------------------- scores
