@@ -39,7 +39,6 @@ from block_sparse_attention_12_b200 import inputs, multigpu  # noqa: E402
 
 METRIC = "AB-Attn fwd ms & executed TFLOPS (% bf16 TC peak), 75.6K tok × 40 heads"
 UNIT = "TFLOP/s"
-FP32_LANES_PER_SM = 128
 
 
 def parse():
@@ -496,19 +495,23 @@ def main():
     nqb, nkvb = math.ceil(w.N / 128), math.ceil(w.N / w.kv_block)
     rows = BH * nqb
     sel_cnt = float(plan.counts.sum().item())
-    fp32_peak = 148 * FP32_LANES_PER_SM * 2 * P["sm_mhz"] * 1e6 / 1e12
     roofs = {
         "forward": {"bound": "tensor", "achieved": fwd_tf, "peak": P["bf16"], "unit": "TFLOP/s",
                     "work": fwd_fl, "traffic": traffic_for("forward", rows)},
         "meanpool": {"bound": "hbm", "unit": "GB/s", "peak": P["hbm"],
                      "work": BH * w.N * w.d * 2 + BH * nkvb * w.d * 4,
                      "traffic": traffic_for("meanpool", BH * nkvb)},
-        "kmeans": {"bound": "alu", "unit": "TFLOP/s", "peak": fp32_peak,
-                   "work": rows * w.kmeans_iters * (128 * 8 * w.d * 3 + 128 * w.d * 8 * 2),
+        # k-means (both Lloyd steps on tcgen05, 16-column accumulators) is bound by
+        # the latency of its dependent iterations; its roofline is its one read of
+        # the queries (and the centroid, weight and label writes)
+        "kmeans": {"bound": "hbm", "unit": "GB/s", "peak": P["hbm"],
+                   "work": rows * (128 * w.d * 2 + w.n_clusters * w.d * 4 + w.n_clusters * 4 + 128 * 4),
                    "traffic": traffic_for("kmeans", rows)},
         # tensor cores, bf16 hi/lo split: 3 MMAs per product, 2 passes over 8 cluster slots
         "score": {"bound": "tensor", "unit": "TFLOP/s", "peak": P["bf16"],
-                  "work": 3 * 2 * (2.0 * rows * 8 * nkvb * w.d), "traffic": traffic_for("score", rows)},
+                  "work": 3 * 2 * (2.0 * rows * 8 * nkvb * w.d), "traffic": traffic_for("score", rows),
+                  # its HBM side: the mean keys once per head, the centroids, the scores written
+                  "hbm_bytes": BH * nkvb * w.d * 4 + rows * 8 * w.d * 4 + rows * nkvb * 4},
         "planner": {"bound": "hbm", "unit": "GB/s", "peak": P["hbm"],
                     "work": rows * nkvb * 4 + rows * 4 + sel_cnt * 8, "traffic": traffic_for("planner", rows)},
     }
@@ -518,14 +521,15 @@ def main():
             r["achieved"] = r["work"] / t / (1e9 if r["unit"] == "GB/s" else 1e12)
         r["frac"] = r["achieved"] / r["peak"]
         r["ms"] = kb_ms[k]
+        if "hbm_bytes" in r:
+            r["hbm_gbs"] = r["hbm_bytes"] / t / 1e9
+            r["hbm_frac"] = r["hbm_gbs"] / P["hbm"]
     step_share = {k: kb_ms[k] * (w.forwards_per_plan if k == "forward" else 1) for k in roofs}
     dom = max(step_share, key=step_share.get)
     rd = roofs[dom]
     roofline = {"kernel": dom, "bound": rd["bound"], "achieved": rd["achieved"], "peak": rd["peak"],
                 "unit": rd["unit"], "frac": rd["frac"], "traffic": rd["traffic"],
-                "peak_source": P["src"] + (" bf16 burst" if rd["bound"] == "tensor" else
-                                           (" hbm copy" if rd["bound"] == "hbm" else
-                                            " fp32 lanes x 2 x max SM clock (derived)"))}
+                "peak_source": P["src"] + (" bf16 burst" if rd["bound"] == "tensor" else " hbm copy")}
 
     # ---- end to end through the public API with host buffers: every step
     # copies its Q, K, V from pinned host memory and its O back; steps are
