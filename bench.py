@@ -614,7 +614,9 @@ def main():
         "dense": dense, "roofline": roofline,
         "rooflines": {k: {kk: vv for kk, vv in r.items() if kk != "work"} for k, r in roofs.items()},
         "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
-        "gpu_launches": 7 * args.steps if w.forwards_per_plan == 1 else (6 + w.forwards_per_plan) * args.steps,
+        # per step: abattn_plan launches mean keys, k-means, scores and the planner;
+        # then one forward per plan use
+        "gpu_launches": (4 + w.forwards_per_plan) * args.steps,
         "peaks": P,
     }
     print(json.dumps(line), flush=True)
