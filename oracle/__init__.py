@@ -107,12 +107,13 @@ def meanpool(K, kb: int) -> np.ndarray:
 
 
 def kmeans(Qb, nc: int = 8, iters: int = 10):
-    """Qb [M, d] -> (C [nc, d], w [nc], labels [M])."""
+    """Qb [M, d] -> (C [nc, d], w [nc], labels [M]); with no iterations no
+    query is assigned and every label is -1."""
     Qb = f64(Qb)
     M, d = Qb.shape
     C = np.empty((nc, d))
     w = np.empty(nc)
-    lab = np.empty(M, dtype=np.int32)
+    lab = np.full(M, -1, dtype=np.int32)
     lib().oc_kmeans(Qb, M, d, nc, iters, C, w, lab)
     return C, w, lab
 

@@ -99,8 +99,9 @@ def test_kmeans_parity(tiny):
     assert agree_rows >= 0.9 * nrows
 
 
-def test_kmeans_ragged_block_and_few_clusters():
-    N, d = 1000, 128
+@pytest.mark.parametrize("d", [64, 128])
+def test_kmeans_ragged_block_and_few_clusters(d):
+    N = 1000
     Q = torch.randn(1, 2, N, d, generator=torch.Generator().manual_seed(5)).to(torch.bfloat16)
     cfg = abi.Config(n_clusters=5, kmeans_iters=7)
     C, w, lab = abi.kmeans(Q.cuda(), cfg)
@@ -112,6 +113,28 @@ def test_kmeans_ragged_block_and_few_clusters():
     np.testing.assert_array_equal(lg[:N - qb * 128], lo)
     np.testing.assert_allclose(C[0, 1, qb].cpu().numpy(), Co, rtol=1e-5, atol=1e-5)
     np.testing.assert_array_equal(w[0, 1, qb].cpu().numpy(), wo.astype(np.float32))
+
+
+def test_kmeans_degenerate_cases():
+    """No iterations (the initial centroids, equal weights) and a block of
+    identical queries (every distance ties, so every query joins cluster 0)."""
+    N, d = 256, 64
+    g = torch.Generator().manual_seed(9)
+    Q = torch.randn(1, 1, N, d, generator=g).to(torch.bfloat16)
+    Q[0, 0, 128:] = Q[0, 0, 128]
+    C0, w0, lab0 = abi.kmeans(Q.cuda(), abi.Config(kmeans_iters=0))
+    C, w, lab = abi.kmeans(Q.cuda(), abi.Config(kmeans_iters=10))
+    abi.check()
+    for qb in range(2):
+        Co, wo, lo = oracle.kmeans(Q[0, 0, qb * 128:(qb + 1) * 128], 8, 0)
+        np.testing.assert_array_equal(C0[0, 0, qb].cpu().numpy(), Co.astype(np.float32))
+        np.testing.assert_array_equal(w0[0, 0, qb].cpu().numpy(), wo.astype(np.float32))
+        np.testing.assert_array_equal(lab0[0, 0, qb].cpu().numpy(), lo)  # -1: no query assigned
+    Co, wo, lo = oracle.kmeans(Q[0, 0, 128:], 8, 10)
+    np.testing.assert_array_equal(lab[0, 0, 1].cpu().numpy(), lo)
+    assert np.all(lo == 0) and wo[0] == 1.0
+    np.testing.assert_array_equal(w[0, 0, 1].cpu().numpy(), wo.astype(np.float32))
+    np.testing.assert_allclose(C[0, 0, 1].cpu().numpy(), Co, rtol=1e-6, atol=1e-6)
 
 
 def test_score_parity_fed_inputs(tiny):
