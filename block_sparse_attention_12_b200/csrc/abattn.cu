@@ -281,7 +281,7 @@ int run_forward(bool dense, const void *Q, const void *K, const void *V, const a
     int rc = check_device();
     if (rc) return rc;
     CUtensorMap mQ, mK, mV;
-    const int box = dense ? 32 : (kb < 32 ? kb : 32);
+    const int box = 32;  // K/V TMA boxes of the dense kernel (the sparse kernel gathers with cp.async)
     if ((rc = make_map(&mQ, Q, d, 128)) || (rc = make_map(&mK, K, d, box)) || (rc = make_map(&mV, V, d, box)))
         return rc;
     FwdParams fp;

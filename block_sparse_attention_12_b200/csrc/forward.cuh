@@ -55,7 +55,7 @@ constexpr int FWD_SOFTMAX_REGS = ABATTN_FWD_SOFTMAX_REGS;
 constexpr int FWD_OTHER_REGS = ABATTN_FWD_OTHER_REGS;
 static_assert(2 * 128 * FWD_SOFTMAX_REGS + 2 * 128 * FWD_OTHER_REGS <= FWD_THREADS * 128,
               "setmaxnreg split exceeds the launch register budget");
-constexpr int FWD_PRODUCERS = 7;  // producer warps (8..11, 13..15); warp w owns the tile's block slots = w mod 7
+constexpr int FWD_PRODUCERS = 7;  // producer warps (8..11, 13..15); producer w gathers the quads q = w mod 7 of a tile
 constexpr int FWD_NS = 3;  // K/V stages
 // O and the row sum are rescaled only when a tile's max exceeds the running
 // reference max by more than this (log2 units).  Probabilities then stay
@@ -80,7 +80,7 @@ struct FwdParams {
     int N;
     int nqb;
     int kb;
-    int box_rows;  // rows per K/V TMA box: min(kb, 32)
+    int box_rows;  // dense kernel: rows per K/V TMA box (32)
     int nkvb;
     float scale_log2;
 };
