@@ -150,8 +150,9 @@ __device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t *bar) {
 
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-// Makes this thread's generic-proxy shared-memory writes visible to the
-// async proxy (tensor-core operand reads).
+// Proxy fence: orders the generic-proxy shared-memory writes this thread has
+// made, or has observed through a barrier it acquired, before its later
+// async-proxy operations (TMA, tensor-core operand reads).
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }

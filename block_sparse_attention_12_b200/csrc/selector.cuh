@@ -104,16 +104,19 @@ __global__ void split_rows_kernel(const float *__restrict__ src, int64_t nblk, i
 // Products are exact (bf16 x bf16, or x 0/1) and accumulate in fp32.  An
 // empty cluster keeps its centroid; a fixed point (no label moved) ends the
 // iterations early with the same result.  For d = 64 the tile's second
-// 64-column half is zero, so the update still has M = 128 rows.
+// 64-column half is zero, so the update still has M = 128 rows.  Thread k
+// keeps the fp32 centroids of dimension k in registers, and the one-hot
+// operand shares its tile with the centroids' lo part (the assignment has
+// read that before the one-hot is written, the update has read the one-hot
+// before the new centroids are), so five CTAs fit an SM.
 constexpr int KM_THREADS = 128;
 
 struct KmLayout {
     static constexpr int Q_OFF = 0;          // [2 halves][128 rows][128 B]
     static constexpr int CHI_OFF = 32768;    // [2 halves][16 rows][128 B]
-    static constexpr int CLO_OFF = 36864;
-    static constexpr int OH_OFF = 40960;     // one-hot, [2 query halves][16 rows][128 B]
-    static constexpr int CS_OFF = 45056;     // fp32 centroids [8][128]
-    static constexpr int CN_OFF = CS_OFF + 8 * 128 * 4;  // |c|^2 [8], partials [4][8]
+    static constexpr int CLO_OFF = 36864;    // the same, or the one-hot [2 query halves][16 rows][128 B]
+    static constexpr int OH_OFF = CLO_OFF;
+    static constexpr int CN_OFF = CLO_OFF + 4096;        // |c|^2 [8], partials [4][8]
     static constexpr int INT_OFF = CN_OFF + 40 * 4;      // lab[128], cnt[8], wcnt[4][8]
     static constexpr int BAR_OFF = INT_OFF + (128 + 8 + 32) * 4;  // q_bar, mma_bar
     static constexpr int MISC_OFF = BAR_OFF + 16;         // tmem slot
@@ -129,7 +132,7 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int k, uint32_t hs) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(KM_THREADS) kmeans_kernel(
+__global__ void __launch_bounds__(KM_THREADS, 5) kmeans_kernel(
     const __grid_constant__ CUtensorMap tmQ, int64_t N, int64_t nqb, int nc, int iters,
     float *__restrict__ Cout, float *__restrict__ wout, int32_t *__restrict__ labels_out,
     __nv_bfloat16 *__restrict__ Chi, __nv_bfloat16 *__restrict__ Clo) {
@@ -138,7 +141,6 @@ __global__ void __launch_bounds__(KM_THREADS) kmeans_kernel(
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(km_smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sQ = smem + L::Q_OFF;
     uint8_t *sChi = smem + L::CHI_OFF, *sClo = smem + L::CLO_OFF, *sOH = smem + L::OH_OFF;
-    float *Cs = reinterpret_cast<float *>(smem + L::CS_OFF);   // [8][D]
     float *cn = reinterpret_cast<float *>(smem + L::CN_OFF);   // [8]
     float *cn_part = cn + 8;                                    // [4][8]
     int *lab = reinterpret_cast<int *>(smem + L::INT_OFF);     // [128]
@@ -169,7 +171,7 @@ __global__ void __launch_bounds__(KM_THREADS) kmeans_kernel(
     // and, for d = 64, the tile's second half
     {
         uint4 *z = reinterpret_cast<uint4 *>(smem + L::CHI_OFF);
-        for (int e = tid; e < (3 * 4096) / 16; e += KM_THREADS) z[e] = make_uint4(0, 0, 0, 0);
+        for (int e = tid; e < (2 * 4096) / 16; e += KM_THREADS) z[e] = make_uint4(0, 0, 0, 0);
         if (D == 64) {
             uint4 *zq = reinterpret_cast<uint4 *>(sQ + 16384);
             for (int e = tid; e < 16384 / 16; e += KM_THREADS) zq[e] = make_uint4(0, 0, 0, 0);
@@ -193,10 +195,11 @@ __global__ void __launch_bounds__(KM_THREADS) kmeans_kernel(
     auto qval = [&](int r, int k) {
         return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sQ + sw128_off(r, k, 16384)));
     };
-    // centroid c of dimension k (thread k) into Cs and the bf16 hi/lo operand
+    float cs[8];  // thread k < D: the fp32 centroids' dimension k
+    // centroid c of dimension k (thread k) into cs and the bf16 hi/lo operand
     // tiles; returns its square for |c|^2
     auto set_centroid = [&](int c, int k, float v) {
-        Cs[c * D + k] = v;
+        cs[c] = v;
         __nv_bfloat16 hi, lo;
         split_bf16(v, hi, lo);
         const uint32_t o = sw128_off(c, k, 2048);
@@ -307,7 +310,7 @@ __global__ void __launch_bounds__(KM_THREADS) kmeans_kernel(
             part[c] = 0.f;
             if (tid < D) {
                 const int n = cnt_s[c];
-                const float v = (c < nc && n > 0) ? __uint_as_float(s16[c]) / float(n) : Cs[c * D + tid];
+                const float v = (c < nc && n > 0) ? __uint_as_float(s16[c]) / float(n) : cs[c];
                 part[c] = set_centroid(c, tid, v);
             }
         }
@@ -316,13 +319,14 @@ __global__ void __launch_bounds__(KM_THREADS) kmeans_kernel(
     }
     __syncthreads();
 
-    if (Cout != nullptr)
-        for (int e = tid; e < nc * D; e += KM_THREADS) Cout[row * nc * D + e] = Cs[e];
-    if (Chi != nullptr)  // [rows][8][D], clusters past nc zero
-        for (int e = tid; e < 8 * D; e += KM_THREADS) {
-            const int c = e / D;
-            split_bf16(c < nc ? Cs[e] : 0.f, Chi[row * 8 * D + e], Clo[row * 8 * D + e]);
+    if (tid < D) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            if (Cout != nullptr && c < nc) Cout[(row * nc + c) * D + tid] = cs[c];
+            if (Chi != nullptr)  // [rows][8][D], clusters past nc zero
+                split_bf16(c < nc ? cs[c] : 0.f, Chi[(row * 8 + c) * D + tid], Clo[(row * 8 + c) * D + tid]);
         }
+    }
     if (tid < nc) wout[row * nc + tid] = iters > 0 ? float(cnt_s[tid]) / float(M) : 1.f / float(nc);
     if (labels_out != nullptr)
         labels_out[row * 128 + tid] = (iters > 0 && tid < M) ? lab[tid] : -1;
