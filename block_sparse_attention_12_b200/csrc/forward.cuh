@@ -17,7 +17,10 @@
 //               running max with lazy O rescaling (only when the max grows by
 //               more than 2^32); P = exp2(t - m), packed to bf16 as it is
 //               computed and stored back to TMEM over the first 64 columns of
-//               its S buffer.  At the end the two partial softmaxes are merged
+//               its S buffer (the dense kernel hands keys 0..63 of P to the
+//               MMA warp before it computes the exponentials of keys 64..127,
+//               so that half of PV starts early).  At the end the two partial
+//               softmaxes are merged
 //               (max, sums, O) and O (bf16) and the natural-log LSE are written;
 //   warps 8..11, 13..15  producers (setmaxnreg lowered): warp 8 loads the Q
 //               tile once by TMA.  Sparse kernel: the 32 quads of 4 rows of a
@@ -97,7 +100,7 @@ struct FwdLayout {
     static constexpr int BIAS_OFF = V_OFF + FWD_NS * TILE;
     static constexpr int GBIAS_OFF = BIAS_OFF;
     static constexpr int BAR_OFF = BIAS_OFF + FWD_NS * 128 * 4;
-    static constexpr int NBARS = 1 + 2 * FWD_NS + 6;
+    static constexpr int NBARS = 1 + 2 * FWD_NS + 8;
     // (m, l) of both softmax warpgroups, [2][2][128] floats, exchanged in the
     // epilogue through the first K stage: by then every QK^T MMA has completed
     // and every K load has landed
@@ -128,8 +131,8 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
     uint64_t *kv_full = bars + 1;
     uint64_t *kv_empty = bars + 1 + FWD_NS;
     uint64_t *s_full = bars + 1 + 2 * FWD_NS;  // [2]
-    uint64_t *p_full = s_full + 2;              // [2]
-    uint64_t *pv_done = p_full + 2;             // [2]
+    uint64_t *p_full = s_full + 2;              // [2 warpgroups][2 key halves]
+    uint64_t *pv_done = p_full + 4;             // [2]
     float *xch = reinterpret_cast<float *>(smem + L::XCH_OFF);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::MISC_OFF);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::MISC_OFF + 4);
@@ -160,7 +163,8 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1);
-            mbar_init(&p_full[i], 4);
+            mbar_init(&p_full[2 * i], 4);
+            mbar_init(&p_full[2 * i + 1], 4);
             mbar_init(&pv_done[i], 1);
         }
         *abort_flag = 0;
@@ -374,16 +378,34 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
             for (int t = 0; ok && t < T; ++t) {
                 if (t + 1 < T && !issue_qk(t + 1)) break;
                 const int g = t & 1;  // softmax warpgroup / S buffer / O accumulator of this tile
-                if (!mbar_wait(&p_full[g], (t >> 1) & 1, abort_flag)) break;
-                tc_fence_after();
                 const int s = t % FWD_NS;
                 const uint32_t vb_lo = v_lo + uint32_t(s) * (L::TILE >> 4);
                 const uint32_t pbase = tmem + g * 128;
                 const uint32_t acc0 = t >= 2 ? 1u : 0u;
+                if constexpr (DENSE) {
+                    // PV in two key halves: the softmax releases keys 0..63 of P
+                    // before it computes the exponentials of keys 64..127
+                    bool got = true;
 #pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    umma_ts_lo(tmem + FWD_TMEM_O + g * 128, pbase + k * 8, vb_lo + k * (2048 >> 4), idesc_pv,
-                               k > 0 ? 1u : acc0);
+                    for (int hh = 0; hh < 2; ++hh) {
+                        if (!mbar_wait(&p_full[2 * g + hh], (t >> 1) & 1, abort_flag)) { got = false; break; }
+                        tc_fence_after();
+#pragma unroll
+                        for (int k = 4 * hh; k < 4 * hh + 4; ++k)
+                            umma_ts_lo(tmem + FWD_TMEM_O + g * 128, pbase + k * 8, vb_lo + k * (2048 >> 4),
+                                       idesc_pv, k > 0 ? 1u : acc0);
+                    }
+                    if (!got) break;
+                } else {
+                    // one release of the whole P row (the split measured no
+                    // gain on the sparse kernel)
+                    if (!mbar_wait(&p_full[2 * g + 1], (t >> 1) & 1, abort_flag)) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        umma_ts_lo(tmem + FWD_TMEM_O + g * 128, pbase + k * 8, vb_lo + k * (2048 >> 4), idesc_pv,
+                                   k > 0 ? 1u : acc0);
+                }
                 umma_commit(&kv_empty[s]);
                 umma_commit(&pv_done[g]);
             }
@@ -483,10 +505,11 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                 }
                 return fmaxf(mt0, mt1);
             };
-            // P = 2^(logit - m_ref) into pk, and the row sum
-            auto exp_pass = [&](float m_ref) {
+            // P = 2^(logit - m_ref) into pk for the groups [qa, qa+16) (keys
+            // 4qa .. 4qa+63), and the row sum
+            auto exp_pass = [&](float m_ref, int qa) {
 #pragma unroll
-                for (int q0 = 0; q0 < 32; q0 += 4) {
+                for (int q0 = qa; q0 < qa + 16; q0 += 4) {
                     float4 g4;
                     if constexpr (GROUPED) g4 = *reinterpret_cast<const float4 *>(gbias + q0);
 #pragma unroll
@@ -503,10 +526,17 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                     }
                 }
             };
-            // P row -> TMEM over the first 64 columns of this S buffer
-            auto store_p = [&]() {
-                tmem_st32(t_S, *reinterpret_cast<const uint32_t(*)[32]>(pk));
-                tmem_st32(t_S + 32, *reinterpret_cast<const uint32_t(*)[32]>(pk + 32));
+            // half hh of the P row (keys 64hh .. 64hh+63) -> TMEM columns
+            // [32hh, 32hh+32) of this S buffer
+            auto store_p = [&](int hh) {
+                tmem_st32(t_S + 32 * hh, *reinterpret_cast<const uint32_t(*)[32]>(pk + 32 * hh));
+            };
+            // this warp's P writes (and O rescaling) done: release half hh
+            auto release_p = [&](int hh) {
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&p_full[2 * g + hh]);
             };
             // Lazy rescaling: O and l keep the reference max m until a tile's
             // max exceeds it by more than FWD_RESCALE_LOG2.
@@ -519,32 +549,53 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                 m = m_new;
             }
             const bool any = __any_sync(0xffffffffu, need);
-            exp_pass(m == -INFINITY ? 0.f : m);
-            store_p();
-            l += (rs01.x + rs01.y) + (rs23.x + rs23.y);
-            if (ntiles > 0 && any) {
+            const bool rescale = ntiles > 0 && any;
+            const float m_ref = m == -INFINITY ? 0.f : m;
+            auto rescale_o = [&]() -> bool {
                 // this warpgroup's O must be complete before it is rescaled
-                // (PV(t) is issued only after p_full below).  Waiting only when
-                // rescaling is safe: PV(t) needs our p_full(t), so the barrier is
-                // never more than one phase past the one waited for.
-                if (!mbar_wait(&pv_done[g], ((t >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
+                // (PV(t) waits for our release of P(t)).  Waiting only when
+                // rescaling is safe: PV(t) needs that release, so the barrier
+                // is never more than one phase past the one waited for.
+                if (!mbar_wait(&pv_done[g], ((t >> 1) - 1) & 1, abort_flag)) return false;
                 tc_fence_after();
-                {
 #pragma unroll
-                    for (int c = 0; c < HD / 32; ++c) {
-                        uint32_t o[32];
-                        tmem_ld32(t_O + c * 32, o);
-                        tmem_wait_ld();
+                for (int c = 0; c < HD / 32; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(t_O + c * 32, o);
+                    tmem_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                        tmem_st32(t_O + c * 32, o);
-                    }
+                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                    tmem_st32(t_O + c * 32, o);
                 }
+                return true;
+            };
+            if constexpr (DENSE) {
+                // keys 0..63 of P go to the MMA warp before the exponentials of
+                // keys 64..127, unless this warp's rows of O are to be rescaled
+                // first (PV(t) must add to the rescaled O)
+                exp_pass(m_ref, 0);
+                if (!rescale) {
+                    store_p(0);
+                    release_p(0);
+                }
+                exp_pass(m_ref, 16);
+                if (rescale) store_p(0);
+                store_p(1);
+                if (rescale) {
+                    if (!rescale_o()) { ok = false; break; }
+                    release_p(0);
+                }
+                release_p(1);
+                l += (rs01.x + rs01.y) + (rs23.x + rs23.y);
+            } else {
+                exp_pass(m_ref, 0);
+                exp_pass(m_ref, 16);
+                store_p(0);
+                store_p(1);
+                l += (rs01.x + rs01.y) + (rs23.x + rs23.y);
+                if (rescale && !rescale_o()) { ok = false; break; }
+                release_p(1);
             }
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&p_full[g]);
         }
         // ------------------------------------------------------------ epilogue
         // wait for this warpgroup's last PV, swap (m, l) with the other
