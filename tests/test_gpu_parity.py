@@ -378,6 +378,40 @@ def test_full_plan_equals_dense(tiny):
     np.testing.assert_allclose(ls.cpu().numpy(), ld.cpu().numpy(), atol=1e-3)
 
 
+def _climbing_logits(N, d, step_log2=40.0, seed=0):
+    """Q, K, V in bf16 whose scaled logits (log2 units) climb by about
+    step_log2 per 128-key tile for the first 64 queries of every q-block: each
+    tile raises those rows' running max by more than the forward's lazy
+    rescale threshold (a factor 2^32), so their O is rescaled at every tile.
+    The other 64 queries see logits of a few units and never rescale, so one
+    warpgroup holds warps on both paths."""
+    g = torch.Generator().manual_seed(seed)
+    Q = 0.05 * torch.randn(1, 1, N, d, generator=g)
+    K = 0.5 * torch.randn(1, 1, N, d, generator=g)
+    V = torch.randn(1, 1, N, d, generator=g)
+    Q[0, 0, (torch.arange(N) % 128) < 64, 0] = 8.0
+    tile = (torch.arange(N) // 128).double()
+    K[0, 0, :, 0] = (step_log2 * tile * math.sqrt(d) / (8.0 * math.log2(math.e))
+                     + 0.5 * torch.randn(N, generator=g, dtype=torch.float64)).float()
+    return tuple(t.to(torch.bfloat16) for t in (Q, K, V))
+
+
+# N % 4 == 0: per-group bias path of the sparse kernel; otherwise per key
+@pytest.mark.parametrize("d,N", [(128, 1024), (64, 1000), (128, 1001)])
+def test_lazy_rescale_on_climbing_logits(d, N):
+    Qc, Kc, Vc = _climbing_logits(N, d)
+    Q, K, V = Qc.cuda(), Kc.cuda(), Vc.cuda()
+    Oo, lo = oracle.dense(Qc[0, 0], Kc[0, 0], Vc[0, 0], 1 / math.sqrt(d))
+    assert lo[:64].max() > 100.0  # the climbing rows reach logits far past the threshold
+    Od, ld = abi.dense_forward(Q, K, V)
+    plan = abi.full_plan(tuple(Q.shape), 4)
+    Os, ls = abi.forward(Q, K, V, plan, abi.Config(kv_block=4))
+    abi.check()
+    for O, lse, what in ((Od, ld, "dense"), (Os, ls, "sparse, full plan")):
+        assert_forward_close(O[0, 0].float().cpu().numpy(), Oo, f"{what} d{d} N{N}")
+        np.testing.assert_allclose(lse[0, 0].cpu().numpy(), lo, atol=2e-3, rtol=1e-4, err_msg=what)
+
+
 # N % 4 == 0 takes the kernel's per-group bias path, the rest its per-key path
 @pytest.mark.parametrize("d,N,kb,budget", [(128, 1000, 4, 0.2), (128, 300, 128, 0.5), (64, 777, 128, 1.0),
                                            (128, 640, 16, 0.3), (64, 2048, 8, 0.1), (128, 1234, 4, 0.25),
