@@ -378,6 +378,45 @@ def test_full_plan_equals_dense(tiny):
     np.testing.assert_allclose(ls.cpu().numpy(), ld.cpu().numpy(), atol=1e-3)
 
 
+def test_batch_of_two_indexes_rows_by_batch():
+    """B = 2 (every workload above has B = 1): each stage indexes its rows as
+    (b, h, qb) and the plan's Philox counter carries b.  Mean keys, k-means and
+    scores (fed the oracle's inputs) against the oracle; the plan bit for bit
+    from the oracle's pi; the forward against the oracle on the GPU's plan."""
+    B, H, N, d, kb = 2, 2, 1000, 128, 4
+    g = torch.Generator().manual_seed(11)
+    Qc, Kc, Vc = (torch.randn(B, H, N, d, generator=g).to(torch.bfloat16) for _ in range(3))
+    cfg = abi.Config(kv_block=kb, budget=0.2, seed=5)
+    Q, K, V = Qc.cuda(), Kc.cuda(), Vc.cuda()
+    shape, scale = (B, H, N, d), 1 / math.sqrt(d)
+    sel = oracle.selector_all(Qc, Kc, 128, kb, cfg.n_clusters, cfg.kmeans_iters, scale)
+    Kb = abi.meanpool(K, kb)
+    C, w, lab = abi.kmeans(Q, cfg)
+    abi.check()
+    np.testing.assert_allclose(Kb.cpu().numpy(), sel["Kbar"], rtol=1e-6, atol=1e-6)
+    assert (lab.cpu().numpy() == sel["labels"]).mean() >= 0.99
+    C32, w32, K32 = (torch.from_numpy(sel[k]).float() for k in ("C", "w", "Kbar"))
+    Sg = abi.score(C32.cuda(), w32.cuda(), K32.cuda(), shape, cfg).cpu().numpy()
+    abi.check()
+    for b, h, qb in np.ndindex(B, H, 8):
+        so = oracle.scores(C32[b, h, qb].double(), w32[b, h, qb].double(), K32[b, h].double(), scale)
+        assert_scores_close(Sg[b, h, qb], so)
+    po = oracle.plan_all(sel["S"], cfg.budget, 0, cfg.seed, want_pi=True)
+    pg = abi.plan_from_pi(torch.from_numpy(po["pi"]).cuda(), shape, cfg)
+    abi.check()
+    cg, ig, sg = pg.counts.cpu().numpy(), pg.idx.cpu().numpy(), pg.pi_sel.cpu().numpy()
+    np.testing.assert_array_equal(cg, po["counts"])
+    for r in np.ndindex(cg.shape):
+        np.testing.assert_array_equal(ig[r][:cg[r]], po["idx"][r][:cg[r]])
+        np.testing.assert_array_equal(sg[r][:cg[r]], po["pi_sel"][r][:cg[r]])
+    plan = abi.plan(Q, K, cfg)
+    O, lse = abi.forward(Q, K, V, plan, cfg)
+    abi.check()
+    Oo, lo = _oracle_forward(Qc, Kc, Vc, plan, kb)
+    assert_forward_close(O.float().cpu().numpy(), Oo, "B = 2")
+    np.testing.assert_allclose(lse.cpu().numpy(), lo, atol=2e-3, rtol=1e-4)
+
+
 def _climbing_logits(N, d, step_log2=40.0, seed=0):
     """Q, K, V in bf16 whose scaled logits (log2 units) climb by about
     step_log2 per 128-key tile for the first 64 queries of every q-block: each
