@@ -1,4 +1,5 @@
-"""Builds libabattn.so in-tree with nvcc for sm_100a (B200)."""
+"""Builds libabattn.so, and the self-test library libabattn_selftest.so,
+in-tree with nvcc for sm_100a (B200)."""
 from __future__ import annotations
 
 import glob
@@ -9,6 +10,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libabattn.so")
+SELFTEST_SRC = os.path.join(HERE, "selftest", "wait_selftest.cu")
+SELFTEST_LIB = os.path.join(HERE, "libabattn_selftest.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 FLAGS = [
@@ -24,22 +27,40 @@ def sources():
                   + [os.path.join(ROOT, "include", "abattn.h")])
 
 
-def stale() -> bool:
-    if not os.path.exists(LIB):
+def selftest_sources():
+    return [SELFTEST_SRC, os.path.join(CSRC, "common.cuh"), os.path.join(ROOT, "include", "abattn.h"),
+            os.path.join(ROOT, "include", "abattn_selftest.h")]
+
+
+def stale(lib: str = LIB, srcs=None) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
-    return any(os.path.getmtime(s) > t for s in sources())
+    t = os.path.getmtime(lib)
+    return any(os.path.getmtime(s) > t for s in (sources() if srcs is None else srcs))
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not stale():
-        return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [NVCC, *FLAGS, "-o", tmp, os.path.join(CSRC, "abattn.cu")]
+def _nvcc(src: str, lib: str, verbose: bool, extra=()) -> None:
+    tmp = lib + f".tmp{os.getpid()}"
+    cmd = [NVCC, *FLAGS, *extra, "-o", tmp, src]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
+    os.replace(tmp, lib)
+
+
+def build_selftest(force: bool = False, verbose: bool = False) -> str:
+    if force or stale(SELFTEST_LIB, selftest_sources()):
+        # hidden symbols: its copy of the device error word never binds to
+        # libabattn.so's, however the two libraries are loaded
+        _nvcc(SELFTEST_SRC, SELFTEST_LIB, verbose, ["-Xcompiler", "-fvisibility=hidden"])
+    return SELFTEST_LIB
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    """Builds both libraries (each only when stale); returns libabattn.so."""
+    if force or stale():
+        _nvcc(os.path.join(CSRC, "abattn.cu"), LIB, verbose)
+    build_selftest(force, verbose)
     return LIB
 
 

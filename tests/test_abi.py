@@ -129,3 +129,16 @@ def test_params_struct_layout_matches_header():
     assert abi.Params.seed.offset == 24 and abi.Params.scale.offset == 32
     assert abi.Params.head_offset.offset == 36
     assert ctypes.sizeof(abi.Dims) == 32
+
+
+def test_selftest_library_declares_exports_and_rejects_null():
+    """The failure-detection self-test library (include/abattn_selftest.h)
+    builds, exports exactly what its header declares, and refuses a NULL
+    output pointer on the host, before any CUDA call."""
+    text = open(os.path.join(ROOT, "include", "abattn_selftest.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    assert sorted(set(re.findall(r"\b(abattn_[a-z_]+)\s*\(", text))) == ["abattn_selftest_stalled_wait"]
+    S = ctypes.CDLL(build.build_selftest())
+    f = S.abattn_selftest_stalled_wait
+    f.restype, f.argtypes = ctypes.c_int, [ctypes.POINTER(ctypes.c_int), ctypes.c_void_p]
+    assert f(None, None) == abi.ERR_NULL
