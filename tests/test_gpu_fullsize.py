@@ -15,11 +15,16 @@ Per sampled row:
     the GPU's pi bit for bit;
   * the forward output matches the oracle's forward on the GPU's plan within
     max-abs 2e-2 and relative-L2 5e-3.  The max-abs bound is stated for
-    unit-scale values: it is taken on |error| / max(1, |O|) (a bf16 output
-    above 4 is itself rounded by more than 2e-2) and, on the 14B-like layer
-    whose outlier tokens are scaled x8, in units of that scale (the bf16
-    P.V error grows with |V|).  The relative-L2 bound is scale-free and
-    applies unchanged.
+    unit-scale values and applied per element through the error model of
+    the kernel's P.V product: P is rounded to bf16 (relative error <= 2^-9)
+    before it multiplies V, so the error of output element (i, c) is bounded
+    by 2^-9 * A_ic with A_ic = sum_t p_it |v_tc|, the same softmax weights
+    applied to |V| (the oracle's forward with |V| in place of V).  The bound
+    is |error_ic| <= 2e-2 * max(1, A_ic): the plain absolute 2e-2 wherever
+    A <= 1, scaled only where the row draws on large values (the 14B-like
+    layer's x8 outlier tokens).  The layers without outliers are also held
+    to the plain bound on |error| / max(1, |O|).  The relative-L2 bound is
+    scale-free and applies unchanged.
 """
 import dataclasses
 import math
@@ -36,11 +41,20 @@ pytestmark = pytest.mark.gpu
 WORKLOADS = [inputs.WAN_1_3B, inputs.WAN_14B, inputs.HUNYUAN]
 
 
-def input_scale(w):
-    """Scale of the layer's inputs in units of the unit-variance tokens: the
-    14B-like layer multiplies 1% of its tokens by 8, and the error of the
-    bf16 P.V product grows with |V|."""
-    return w.outlier_scale if w.outlier_frac > 0 else 1.0
+def check_forward(w, Og, Oo, Ao, what):
+    """Max-abs 2e-2 per element on |error| / max(1, A) with A the oracle's
+    forward on |V| (the bf16-P error model), the plain |error| / max(1, |O|)
+    on layers without outlier tokens, and relative-L2 5e-3.  Prints the
+    unscaled error so each layer's margin is on record."""
+    e = np.abs(Og - Oo)
+    err_a = (e / np.maximum(1.0, Ao)).max()
+    err_o = (e / np.maximum(1.0, np.abs(Oo))).max()
+    rel = np.linalg.norm(Og - Oo) / np.linalg.norm(Oo)
+    print(f"{w.name} {what}: max|err| {e.max():.3e} (max A {Ao.max():.2f}), "
+          f"err/max(1,A) {err_a:.3e}, err/max(1,|O|) {err_o:.3e}, rel-L2 {rel:.3e}")
+    assert err_a <= 2e-2 and rel <= 5e-3, (what, err_a, rel)
+    if w.outlier_frac == 0:
+        assert err_o <= 2e-2, (what, err_o)
 
 
 def _cfg(w, **kw):
@@ -132,10 +146,9 @@ def test_sampled_rows_against_oracle(layer):
         np.testing.assert_array_equal(plan.pi_sel[b, h, qb, :n].cpu().numpy(), ps_o)
         # forward on the GPU's plan
         Oo, lo_ = oracle.sparse_block(q[q0:q0 + M], k, v, w.kv_block, idx_o, ps_o, scale)
+        Ao, _ = oracle.sparse_block(q[q0:q0 + M], k, np.abs(v), w.kv_block, idx_o, ps_o, scale)
         Og = O[b, h, q0:q0 + M].float().cpu().numpy().astype(np.float64)
-        err = (np.abs(Og - Oo) / np.maximum(1.0, np.abs(Oo))).max() / input_scale(w)
-        rel = np.linalg.norm(Og - Oo) / np.linalg.norm(Oo)
-        assert err <= 2e-2 and rel <= 5e-3, (h, qb, err, rel)
+        check_forward(w, Og, Oo, Ao, f"sparse row (h {h}, qb {qb})")
         np.testing.assert_allclose(layer["lse"][b, h, q0:q0 + M].cpu().numpy(), lo_, atol=2e-3, rtol=1e-4)
 
 
@@ -165,7 +178,7 @@ def test_dense_rows_against_oracle(layer):
     q, k, v = layer["data"][h]
     for q0 in (0, 128 * 300, w.N - 16):
         Oo, lo = oracle.dense(q[q0:q0 + 16], k, v, 1 / math.sqrt(w.d))
+        Ao, _ = oracle.dense(q[q0:q0 + 16], k, np.abs(v), 1 / math.sqrt(w.d))
         Og = O[0, 0, q0:q0 + 16].float().cpu().numpy().astype(np.float64)
-        assert (np.abs(Og - Oo) / np.maximum(1.0, np.abs(Oo))).max() / input_scale(w) <= 2e-2
-        assert np.linalg.norm(Og - Oo) / np.linalg.norm(Oo) <= 5e-3
+        check_forward(w, Og, Oo, Ao, f"dense rows {q0}..{q0 + 15} (h {h})")
         np.testing.assert_allclose(lse[0, 0, q0:q0 + 16].cpu().numpy(), lo, atol=2e-3, rtol=1e-4)
