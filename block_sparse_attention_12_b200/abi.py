@@ -28,7 +28,22 @@ EXPORTED = [
     "abattn_kmeans", "abattn_score", "abattn_plan_from_scores", "abattn_plan_from_pi",
     "abattn_plan", "abattn_forward", "abattn_dense_forward", "abattn_plan_noalloc",
 ]
-NOALLOC_SCRATCH_BYTES = 32 << 20
+
+
+def _header_define(name: str) -> int:
+    """Integer value of a `#define NAME (a << b)` or `#define NAME n` in
+    include/abattn.h, so that the binding and the library share one value."""
+    import re
+    path = os.path.join(os.path.dirname(_HERE), "include", "abattn.h")
+    with open(path) as f:
+        m = re.search(r"#define\s+" + name + r"\s+\((\d+)u?\s*<<\s*(\d+)\)|#define\s+" + name + r"\s+(\d+)",
+                      f.read())
+    if m is None:
+        raise RuntimeError(f"{name} not found in {path}")
+    return int(m.group(1)) << int(m.group(2)) if m.group(1) else int(m.group(3))
+
+
+NOALLOC_SCRATCH_BYTES = _header_define("ABATTN_NOALLOC_SCRATCH_BYTES")
 
 
 class Dims(ctypes.Structure):

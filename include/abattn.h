@@ -180,8 +180,9 @@ int abattn_dense_forward(const void *Q, const void *K, const void *V, const abat
  *    ABATTN_NOALLOC_SCRATCH_BYTES are rejected with ABATTN_ERR_WORKSPACE
  *    before anything is launched.
  *  - The first call on a device looks up the scratch array's device address
- *    (cudaGetSymbolAddress) with that device current; make that first call
- *    before any stream capture.
+ *    (cudaGetSymbolAddress) with that device current and keeps it for the
+ *    life of the process; make that first call before any stream capture,
+ *    and do not reset the device (cudaDeviceReset) after it.
  *  - All calls on a device share the one array and it keeps the last call's
  *    contents (nothing in it needs clearing: every value read is written
  *    earlier in the same call).  Calls that overlap on the GPU, e.g. on two

@@ -1,6 +1,7 @@
-"""The benchmark's reference arm (the CPU oracle on sampled rows) keeps the
-JSON-line contract the harness parses, and under a multi-rank
-launch only rank 0 prints.  CPU only: the reference arm never touches a GPU."""
+"""The benchmark's reference arm (the CPU oracle on sampled rows) prints
+one well-formed JSON line with the keys a reader of the benchmark output
+expects, and under a multi-rank launch only rank 0 prints.  CPU only: the
+reference arm never touches a GPU."""
 import json
 import os
 import subprocess

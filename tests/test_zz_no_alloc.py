@@ -20,11 +20,19 @@ from block_sparse_attention_12_b200 import abi, inputs
 def test_noalloc_rejects_problems_larger_than_its_scratch():
     shape = (1, 40, 75600, 128)
     cfg = abi.Config(kv_block=4, budget=0.08)
+    # the binding's limit is read from the header the library is built from
+    assert abi.NOALLOC_SCRATCH_BYTES == abi._header_define("ABATTN_NOALLOC_SCRATCH_BYTES") == 32 << 20
     assert abi.plan_workspace_bytes(shape, cfg) > abi.NOALLOC_SCRATCH_BYTES
-    fake = ctypes.c_void_p(0x10000)  # never dereferenced: the size check comes first
-    rc = abi.lib().abattn_plan_noalloc(fake, fake, ctypes.byref(abi.Dims(*shape)), ctypes.byref(cfg.params()),
-                                       fake, fake, fake, abi.capacity(shape, cfg), None)
+    # NULL tensors: whichever check comes first, nothing can be launched on them
+    rc = abi.lib().abattn_plan_noalloc(None, None, ctypes.byref(abi.Dims(*shape)), ctypes.byref(cfg.params()),
+                                       None, None, None, abi.capacity(shape, cfg), None)
     assert rc == abi.ERR_WORKSPACE
+    # a problem that fits gets past the size check and stops at the NULL pointers
+    small = (1, 2, 4096, 64)
+    assert abi.plan_workspace_bytes(small, cfg) <= abi.NOALLOC_SCRATCH_BYTES
+    rc = abi.lib().abattn_plan_noalloc(None, None, ctypes.byref(abi.Dims(*small)), ctypes.byref(cfg.params()),
+                                       None, None, None, abi.capacity(small, cfg), None)
+    assert rc == abi.ERR_NULL
 
 
 @pytest.mark.gpu
