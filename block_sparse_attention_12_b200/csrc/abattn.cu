@@ -519,7 +519,9 @@ int abattn_dense_forward(const void *Q, const void *K, const void *V, const abat
 // library, for callers that may not allocate device memory themselves.
 namespace {
 
-constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB per device, held until exit
+// 32 MiB per device, held until exit; the size is the header's, so the C
+// limit and the documented one cannot drift apart
+constexpr size_t kNoAllocScratchBytes = size_t(ABATTN_NOALLOC_SCRATCH_BYTES);
 
 static __device__ __align__(256) unsigned char g_plan_scratch[kNoAllocScratchBytes];
 
@@ -529,7 +531,9 @@ void *g_scratch_addr[kMaxDevices] = {};
 
 // Device address of g_plan_scratch on the current device.  The name of the
 // array is only a host-side stand-in; the address comes from
-// cudaGetSymbolAddress, looked up once per device with that device current.
+// cudaGetSymbolAddress, looked up once per device with that device current
+// and kept for the life of the process (a cudaDeviceReset after the first
+// call would leave it stale, which the header rules out).
 int scratch_address(void **out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
