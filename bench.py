@@ -53,6 +53,7 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=6)
     ap.add_argument("--dense-iters", type=int, default=3)
     ap.add_argument("--cpu-rows", type=int, default=64)
+    ap.add_argument("--cpu-rows-one-core", type=int, default=12)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -63,6 +64,8 @@ def parse():
     ap.add_argument("--model-layers", type=int, default=40)
     ap.add_argument("--strong", action="store_true",
                     help="one layer's heads sharded over the ranks (head_offset plans, all-gather of O)")
+    ap.add_argument("--gather-bench", action="store_true",
+                    help="microbenchmark of the sparse forward's gather: cp.async, 4-row TMA boxes, TMA gather4")
     ap.add_argument("--sweep", action="store_true",
                     help="budget x kv_block x (SIP, top-k) sweep on the sweep-75k layer, one JSON line per point")
     return ap.parse_args()
@@ -94,7 +97,7 @@ class ClockSampler:
             pass
         try:
             self.p = subprocess.Popen(["nvidia-smi", *sel, f"--query-gpu={self.FIELDS}",
-                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                       "--format=csv,noheader,nounits", "-lms", "50"],
                                       stdout=self.f, stderr=subprocess.DEVNULL)
         except OSError:
             self.p = None
@@ -183,14 +186,26 @@ def run_oracle_rows(w, rows, data, threads: int):
     return time.perf_counter() - t0, flops
 
 
-def cpu_baseline(w, n_rows: int):
+def cpu_baseline(w, n_rows: int, n_rows_one: int):
+    """The oracle on a bounded seeded sample of the workload's rows, on all
+    host cores and on one core.  Rows are independent and their work is
+    proportional to their selected blocks, so the whole layer's time is
+    extrapolated linearly from each sample (reported as such)."""
     threads = os.cpu_count() or 1
+    total_rows = w.B * w.H * math.ceil(w.N / 128)
     rows, data = oracle_sample(w, n_rows)
     secs, flops = run_oracle_rows(w, rows, data, threads)
+    rows1, data1 = oracle_sample(w, n_rows_one, seed_offset=1)
+    secs1, flops1 = run_oracle_rows(w, rows1, data1, 1)
     return {"value": flops / secs / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": f"{len(rows)} (head, q-block) rows of {w.name} (of {w.B * w.H * math.ceil(w.N / 128)}), "
+            "sample": f"{len(rows)} (head, q-block) rows of {w.name} (of {total_rows}), "
                       f"k-means + scores + water-fill + sampling + gathered forward in fp64, "
-                      f"{secs:.2f} s wall on {threads} threads"}
+                      f"{secs:.2f} s wall on {threads} threads",
+            "one_core": {"value": flops1 / secs1 / 1e12, "unit": UNIT, "cores": 1,
+                         "sample": f"{len(rows1)} rows, {secs1:.2f} s on 1 thread"},
+            "extrapolated_layer_ms": {"all_cores": 1e3 * secs * total_rows / len(rows),
+                                      "one_core": 1e3 * secs1 * total_rows / len(rows1),
+                                      "how": "extrapolated: sample time x (layer rows / sampled rows)"}}
 
 
 def run_reference(args, w):
@@ -393,8 +408,40 @@ def run_sweep(args):
                 torch.cuda.empty_cache()
 
 
+def run_gather_bench(args):
+    """Cycles per 128-key tile to gather the 32 selected 4-row blocks of K and
+    V (64 KB) into a 3-stage shared-memory ring, for each copy method and
+    number of issuing warps; one CTA per SM, blocks spread over two heads of
+    75,600 tokens (K and V L2-resident, as in the forward's head-major order).
+    One JSON line per configuration; the microbenchmark also checks the last
+    tile's bytes against global memory."""
+    import ctypes
+    from block_sparse_attention_12_b200 import build
+    lib = ctypes.CDLL(build.build_gatherbench())
+    f = lib.abattn_gather_bench
+    f.argtypes = [ctypes.c_void_p, ctypes.c_void_p] + [ctypes.c_int] * 5 + [
+        ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong)]
+    torch.cuda.set_device(0)
+    BH, N = 2, 75600
+    g = torch.Generator(device="cuda").manual_seed(11)
+    K = torch.randn(BH, N, 128, device="cuda", generator=g).to(torch.bfloat16)
+    V = torch.randn(BH, N, 128, device="cuda", generator=g).to(torch.bfloat16)
+    names = {1: "cp.async 16B/lane", 0: "TMA tiled box 4x64", 2: "TMA tile::gather4"}
+    for mode in (1, 0, 2):
+        for warps in (1, 2, 4, 7, 8, 16):
+            cyc, bad = ctypes.c_double(), ctypes.c_longlong()
+            rc = f(K.data_ptr(), V.data_ptr(), BH, N, mode, warps, 200, ctypes.byref(cyc), ctypes.byref(bad))
+            print(json.dumps({"gather_bench": names[mode], "issuing_warps": warps, "rc": rc,
+                              "cycles_per_tile": cyc.value if rc == 0 else None,
+                              "bytes_per_cycle": 65536 / cyc.value if rc == 0 and cyc.value > 0 else None,
+                              "last_tile_mismatched_chunks": bad.value}), flush=True)
+
+
 def main():
     args = parse()
+    if args.gather_bench:
+        run_gather_bench(args)
+        return
     if args.sweep:
         run_sweep(args)
         return
@@ -590,7 +637,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, args.cpu_rows)
+        cpu = cpu_baseline(w, args.cpu_rows, args.cpu_rows_one_core)
 
     if dist:
         dist.barrier()

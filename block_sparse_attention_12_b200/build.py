@@ -1,5 +1,6 @@
-"""Builds libabattn.so, and the self-test library libabattn_selftest.so,
-in-tree with nvcc for sm_100a (B200)."""
+"""Builds libabattn.so, the self-test library libabattn_selftest.so and the
+gather microbenchmark libabattn_gatherbench.so, in-tree with nvcc for
+sm_100a (B200)."""
 from __future__ import annotations
 
 import glob
@@ -12,6 +13,8 @@ ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libabattn.so")
 SELFTEST_SRC = os.path.join(HERE, "selftest", "wait_selftest.cu")
 SELFTEST_LIB = os.path.join(HERE, "libabattn_selftest.so")
+GATHERBENCH_SRC = os.path.join(HERE, "microbench", "gather_bench.cu")
+GATHERBENCH_LIB = os.path.join(HERE, "libabattn_gatherbench.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 FLAGS = [
@@ -56,11 +59,19 @@ def build_selftest(force: bool = False, verbose: bool = False) -> str:
     return SELFTEST_LIB
 
 
+def build_gatherbench(force: bool = False, verbose: bool = False) -> str:
+    """The gather microbenchmark of the benchmark's --gather-bench mode."""
+    if force or stale(GATHERBENCH_LIB, [GATHERBENCH_SRC]):
+        _nvcc(GATHERBENCH_SRC, GATHERBENCH_LIB, verbose)
+    return GATHERBENCH_LIB
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
-    """Builds both libraries (each only when stale); returns libabattn.so."""
+    """Builds the libraries (each only when stale); returns libabattn.so."""
     if force or stale():
         _nvcc(os.path.join(CSRC, "abattn.cu"), LIB, verbose)
     build_selftest(force, verbose)
+    build_gatherbench(force, verbose)
     return LIB
 
 
