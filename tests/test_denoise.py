@@ -1,11 +1,15 @@
 """Denoising-loop harness: the policy's schedule (CPU) and, on the GPU, that
 every attention call the harness makes equals the same library call made
-directly (dense steps, plan steps, reused plans)."""
+directly (dense steps, plan steps, reused plans), and that a sparse step on a
+reused plan matches the CPU oracle's forward on that plan."""
 import dataclasses
 import math
 
+import numpy as np
 import pytest
 import torch
+
+import oracle
 
 from block_sparse_attention_12_b200 import denoise, inputs
 from block_sparse_attention_12_b200.denoise import DENSE, PLAN_SPARSE, SPARSE, Policy, schedule
@@ -65,6 +69,7 @@ def test_harness_calls_equal_direct_calls():
     L, cfg = res["layers"], res["cfg"]
     sched = schedule(pol, 2)
     last = [None, None]
+    anchored = False
     for t, row in enumerate(sched):
         for lay in L:
             lay.set_step(t)
@@ -82,6 +87,17 @@ def test_harness_calls_equal_direct_calls():
                 assert _same_plan(plan, last[i])
             Os, ls = abi.forward(lay.Q, lay.K, lay.V, plan, cfg)
             assert torch.equal(O, Os) and torch.equal(lse, ls)
+            if a == SPARSE and not anchored:
+                # the oracle's forward on the plan the harness reused, with this
+                # step's activations: max-abs 2e-2 on |err| / max(1, |O|), rel-L2 5e-3
+                Oo, lo = oracle.forward_rows(lay.Q.cpu(), lay.K.cpu(), lay.V.cpu(), 128, w.kv_block,
+                                             plan.counts.cpu().numpy(), plan.idx.cpu().numpy(),
+                                             plan.pi_sel.cpu().numpy(), 1 / math.sqrt(w.d))
+                Og = O.float().cpu().numpy().astype(np.float64)
+                assert (np.abs(Og - Oo) / np.maximum(1.0, np.abs(Oo))).max() <= 2e-2
+                assert np.linalg.norm(Og - Oo) / np.linalg.norm(Oo) <= 5e-3
+                anchored = True
+    assert anchored
     abi.check()
     # (per-call times solved from these tiny, launch-bound steps mean little;
     # the bench reports them on the full-size layers)

@@ -285,7 +285,9 @@ def test_waterfill_fallback_paths():
 def test_head_offset_slices_equal_whole_layer(tiny):
     """A rank holding a slice of the heads plans it with head_offset = the
     slice's first global head: its plan and output equal those rows of the
-    whole layer's (bit for bit), and without the offset the plan differs."""
+    whole layer's (bit for bit), its plan is the oracle's sample of its own pi
+    with the global head index, its forward matches the oracle's, and without
+    the offset the plan differs."""
     cfg = cfg_of(W)
     full = abi.plan(tiny["Q"], tiny["K"], cfg)
     Of, lf = abi.forward(tiny["Q"], tiny["K"], tiny["V"], full, cfg)
@@ -303,6 +305,29 @@ def test_head_offset_slices_equal_whole_layer(tiny):
             assert torch.equal(ps.idx[0, 0, qb, :c], full.idx[0, lo, qb, :c])
             assert torch.equal(ps.pi_sel[0, 0, qb, :c], full.pi_sel[0, lo, qb, :c])
         assert torch.equal(Os[0, 0], Of[0, lo]) and torch.equal(ls[0, 0], lf[0, lo])
+    # the oracle draws with the global head index: the last head's slice,
+    # planned alone with its head_offset, samples exactly the oracle's plan of
+    # the slice's own pi, and its forward on that plan matches the oracle's
+    lo = W.H - 1
+    Qs, Ks, Vs = (t[:, lo:lo + 1].contiguous() for t in (tiny["Q"], tiny["K"], tiny["V"]))
+    cs = cfg_of(W, head_offset=lo)
+    shape_s = tuple(Qs.shape)
+    Kb = abi.meanpool(Ks, W.kv_block)
+    C, wt, _ = abi.kmeans(Qs, cs)
+    S = abi.score(C, wt, Kb, shape_s, cs)
+    pl, pi = abi.plan_from_scores(S, shape_s, cs, want_pi=True)
+    abi.check()
+    pi_np = pi.cpu().numpy()
+    cnt, idx, pss = pl.counts.cpu().numpy(), pl.idx.cpu().numpy(), pl.pi_sel.cpu().numpy()
+    for qb in range(cnt.shape[2]):
+        idx_o, ps_o, n_o = oracle.sample(pi_np[0, 0, qb], W.seed, 0, lo, qb, pl.cap)
+        assert cnt[0, 0, qb] == min(n_o, pl.cap)
+        np.testing.assert_array_equal(idx[0, 0, qb, :cnt[0, 0, qb]], idx_o)
+        np.testing.assert_array_equal(pss[0, 0, qb, :cnt[0, 0, qb]], ps_o)
+    Os, _ = abi.forward(Qs, Ks, Vs, pl, cs)
+    abi.check()
+    Oo, _ = oracle.forward_rows(Qs.cpu(), Ks.cpu(), Vs.cpu(), 128, W.kv_block, cnt, idx, pss, SCALE)
+    assert_forward_close(Os.float().cpu().numpy(), Oo, "head slice")
     # head 1 planned as if it were head 0 draws other uniforms
     p0 = abi.plan(tiny["Q"][:, 1:2].contiguous(), tiny["K"][:, 1:2].contiguous(), cfg_of(W))
     abi.check()
