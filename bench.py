@@ -66,6 +66,8 @@ def parse():
                     help="one layer's heads sharded over the ranks (head_offset plans, all-gather of O)")
     ap.add_argument("--gather-bench", action="store_true",
                     help="microbenchmark of the sparse forward's gather: cp.async, 4-row TMA boxes, TMA gather4")
+    ap.add_argument("--mma-bench", action="store_true",
+                    help="tensor-core rate microbenchmark (cycles per MMA by operand source and N)")
     ap.add_argument("--sweep", action="store_true",
                     help="budget x kv_block x (SIP, top-k) sweep on the sweep-75k layer, one JSON line per point")
     return ap.parse_args()
@@ -437,10 +439,37 @@ def run_gather_bench(args):
                               "last_tile_mismatched_chunks": bad.value}), flush=True)
 
 
+def run_mma_bench(args):
+    """Clock cycles per bf16 tcgen05.mma (M = 128, K = 16) issued back to back
+    by one thread per SM, one CTA per SM: operands in shared memory at N = 64,
+    128 and 256, A in TMEM at N = 128, and the score and forward kernels' own
+    issue patterns.  Full rate is 2*128*N*16 / 8192 cycles per MMA (64 at
+    N = 128).  One JSON line per mode."""
+    import ctypes
+    from block_sparse_attention_12_b200 import build
+    lib = ctypes.CDLL(build.build_mmabench())
+    f = lib.abattn_mma_bench
+    f.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_double)]
+    torch.cuda.set_device(0)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    modes = [(0, "smem A and B, N=128", 128), (1, "smem A and B, N=256", 256), (2, "A in TMEM, N=128", 128),
+             (3, "smem A and B, N=64", 64), (4, "score kernel issue pattern (N=128)", 128),
+             (5, "forward kernel issue pattern (N=128)", 128)]
+    for mode, name, n in modes:
+        cyc = ctypes.c_double()
+        rc = f(mode, 1024, sms, ctypes.byref(cyc))
+        print(json.dumps({"mma_bench": name, "rc": rc, "cycles_per_mma": cyc.value if rc == 0 else None,
+                          "flop_per_cycle_per_sm": 2 * 128 * n * 16 / cyc.value if rc == 0 and cyc.value > 0 else None,
+                          "full_rate_cycles": 2 * 128 * n * 16 / 8192}), flush=True)
+
+
 def main():
     args = parse()
     if args.gather_bench:
         run_gather_bench(args)
+        return
+    if args.mma_bench:
+        run_mma_bench(args)
         return
     if args.sweep:
         run_sweep(args)

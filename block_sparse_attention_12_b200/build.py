@@ -1,6 +1,6 @@
 """Builds libabattn.so, the self-test library libabattn_selftest.so and the
-gather microbenchmark libabattn_gatherbench.so, in-tree with nvcc for
-sm_100a (B200)."""
+gather and MMA-rate microbenchmarks (libabattn_gatherbench.so,
+libabattn_mmabench.so), in-tree with nvcc for sm_100a (B200)."""
 from __future__ import annotations
 
 import glob
@@ -15,6 +15,8 @@ SELFTEST_SRC = os.path.join(HERE, "selftest", "wait_selftest.cu")
 SELFTEST_LIB = os.path.join(HERE, "libabattn_selftest.so")
 GATHERBENCH_SRC = os.path.join(HERE, "microbench", "gather_bench.cu")
 GATHERBENCH_LIB = os.path.join(HERE, "libabattn_gatherbench.so")
+MMABENCH_SRC = os.path.join(HERE, "microbench", "mma_bench.cu")
+MMABENCH_LIB = os.path.join(HERE, "libabattn_mmabench.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 FLAGS = [
@@ -66,12 +68,20 @@ def build_gatherbench(force: bool = False, verbose: bool = False) -> str:
     return GATHERBENCH_LIB
 
 
+def build_mmabench(force: bool = False, verbose: bool = False) -> str:
+    """The tensor-core rate microbenchmark of the benchmark's --mma-bench mode."""
+    if force or stale(MMABENCH_LIB, [MMABENCH_SRC, os.path.join(CSRC, "common.cuh")]):
+        _nvcc(MMABENCH_SRC, MMABENCH_LIB, verbose)
+    return MMABENCH_LIB
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
     """Builds the libraries (each only when stale); returns libabattn.so."""
     if force or stale():
         _nvcc(os.path.join(CSRC, "abattn.cu"), LIB, verbose)
     build_selftest(force, verbose)
     build_gatherbench(force, verbose)
+    build_mmabench(force, verbose)
     return LIB
 
 
