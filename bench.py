@@ -442,25 +442,34 @@ def run_gather_bench(args):
 def run_mma_bench(args):
     """Clock cycles per bf16 tcgen05.mma (M = 128, K = 16) issued back to back
     by one thread per SM, one CTA per SM: operands in shared memory at N = 64,
-    128 and 256, A in TMEM at N = 128, and the score and forward kernels' own
-    issue patterns.  Full rate is 2*128*N*16 / 8192 cycles per MMA (64 at
-    N = 128).  One JSON line per mode."""
+    128 and 256, A in TMEM at N = 128, the score and forward kernels' own
+    issue patterns, and N = 128 beside four warps loading or storing shared
+    memory (with the bytes per cycle those warps get).  Full rate is
+    2*128*N*16 / 8192 cycles per MMA (64 at N = 128).  One JSON line per
+    mode."""
     import ctypes
     from block_sparse_attention_12_b200 import build
     lib = ctypes.CDLL(build.build_mmabench())
     f = lib.abattn_mma_bench
-    f.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_double)]
+    f.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_double),
+                  ctypes.POINTER(ctypes.c_double)]
     torch.cuda.set_device(0)
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     modes = [(0, "smem A and B, N=128", 128), (1, "smem A and B, N=256", 256), (2, "A in TMEM, N=128", 128),
              (3, "smem A and B, N=64", 64), (4, "score kernel issue pattern (N=128)", 128),
-             (5, "forward kernel issue pattern (N=128)", 128)]
+             (5, "forward kernel issue pattern (N=128)", 128),
+             (6, "smem A and B, N=128, 4 warps loading shared memory", 128),
+             (7, "A in TMEM, N=128, 4 warps loading shared memory", 128),
+             (8, "smem A and B, N=128, 4 warps storing shared memory", 128)]
     for mode, name, n in modes:
-        cyc = ctypes.c_double()
-        rc = f(mode, 1024, sms, ctypes.byref(cyc))
-        print(json.dumps({"mma_bench": name, "rc": rc, "cycles_per_mma": cyc.value if rc == 0 else None,
-                          "flop_per_cycle_per_sm": 2 * 128 * n * 16 / cyc.value if rc == 0 and cyc.value > 0 else None,
-                          "full_rate_cycles": 2 * 128 * n * 16 / 8192}), flush=True)
+        cyc, tr = ctypes.c_double(), ctypes.c_double()
+        rc = f(mode, 1024, sms, ctypes.byref(cyc), ctypes.byref(tr))
+        line = {"mma_bench": name, "rc": rc, "cycles_per_mma": cyc.value if rc == 0 else None,
+                "flop_per_cycle_per_sm": 2 * 128 * n * 16 / cyc.value if rc == 0 and cyc.value > 0 else None,
+                "full_rate_cycles": 2 * 128 * n * 16 / 8192}
+        if mode >= 6:
+            line["other_warps_smem_bytes_per_cycle"] = tr.value if rc == 0 else None
+        print(json.dumps(line), flush=True)
 
 
 def main():
