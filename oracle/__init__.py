@@ -281,3 +281,68 @@ def plan_forward_row(Qh, Kh, Vh, Kbar_h, b: int, h: int, qb: int, kb: int, budge
         ps = np.ones(idx.size, dtype=np.float32)
     O, lse = sparse_block(Qb, Kh, Vh, kb, idx, ps, scale)
     return dict(O=O, lse=lse, idx=idx, pi_sel=ps, S=s)
+
+
+# ---------------------------------------------------------------- 8-bit forward inputs
+# The FP8 E4M3 forward (VC-Attention pages, B200 results: 8-bit attention on
+# Blackwell) quantises Q per 128-query block and K per KV block, each block
+# with its own scale.  E4M3 is the OCP 8-bit float with one sign bit, four
+# exponent bits (bias 7) and three mantissa bits; its largest finite value is
+# 448, and there is no infinity.  A block's scale is amax / 448, so that its
+# largest element maps to the largest code; a block of zeros takes scale 1.
+
+E4M3_MAX = 448.0
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """E4M3 byte codes -> float64, from the format definition (NaN for the two
+    NaN codes 0x7F and 0xFF)."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    val = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * 2.0 ** (e - 7))
+    val = sign * val
+    return np.where((c & 0x7F) == 0x7F, np.nan, val)
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """float32 values already inside [-448, 448] -> E4M3 codes, rounded to
+    nearest even (torch's float8_e4m3fn conversion as the rounding step)."""
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(np.asarray(x, dtype=np.float32)))
+    return t.to(torch.float8_e4m3fn).view(torch.uint8).numpy().copy()
+
+
+def quantize_e4m3_rows(X, rows_per_block: int):
+    """X [..., n, d] (the bf16 values as float32) -> (codes uint8 [..., n, d],
+    scales float32 [..., ceil(n / rows_per_block)]).
+
+    Per block of rows_per_block consecutive rows (the last one may be short):
+    amax = max |x| over the block; scale = fp32(amax / 448) and
+    inv = fp32(448 / amax) (1 and 1 for an all-zero block); each element is
+    encoded from fp32(x * inv), clamped to +-448 against the rounding of inv."""
+    X = np.asarray(X, dtype=np.float32)
+    *lead, n, d = X.shape
+    nb = -(-n // rows_per_block)
+    pad = nb * rows_per_block - n
+    Xp = np.concatenate([X, np.zeros((*lead, pad, d), np.float32)], axis=-2) if pad else X
+    blocks = Xp.reshape(*lead, nb, rows_per_block, d)
+    amax = np.abs(blocks).max(axis=(-2, -1))
+    zero = amax == 0
+    safe = np.where(zero, np.float32(1), amax).astype(np.float32)
+    scale = np.where(zero, np.float32(1), (safe / np.float32(E4M3_MAX)).astype(np.float32)).astype(np.float32)
+    inv = np.where(zero, np.float32(1), (np.float32(E4M3_MAX) / safe).astype(np.float32)).astype(np.float32)
+    y = (blocks * inv[..., None, None]).astype(np.float32)
+    y = np.clip(y, -E4M3_MAX, E4M3_MAX).astype(np.float32)
+    codes = e4m3_encode(y).reshape(*lead, nb * rows_per_block, d)[..., :n, :]
+    return np.ascontiguousarray(codes), scale
+
+
+def dequantize_e4m3_rows(codes, scales, rows_per_block: int) -> np.ndarray:
+    """Inverse of quantize_e4m3_rows up to the rounding: code value x block
+    scale, in float64."""
+    v = e4m3_decode(codes)
+    *lead, n, d = v.shape
+    rep = np.repeat(np.asarray(scales, dtype=np.float64), rows_per_block, axis=-1)[..., :n]
+    return v * rep[..., None]
