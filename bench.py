@@ -66,6 +66,8 @@ def parse():
                     help="one layer's heads sharded over the ranks (head_offset plans, all-gather of O)")
     ap.add_argument("--gather-bench", action="store_true",
                     help="microbenchmark of the sparse forward's gather: cp.async, 4-row TMA boxes, TMA gather4")
+    ap.add_argument("--e4m3", action="store_true",
+                    help="the E4M3 forward beside the bf16 forward on the same plan (ms, TFLOP/s, error)")
     ap.add_argument("--mma-bench", action="store_true",
                     help="tensor-core rate microbenchmark (cycles per MMA by operand source and N)")
     ap.add_argument("--sweep", action="store_true",
@@ -410,6 +412,47 @@ def run_sweep(args):
                 torch.cuda.empty_cache()
 
 
+def run_e4m3(args):
+    """The E4M3 forward (QK^T in 8-bit floats, per-block scales) beside the
+    bf16 forward on the same plan of the benchmark's layer: forward ms and
+    executed TFLOP/s of both (CUDA events, inputs larger than L2), the
+    quantisation of Q and K, and the E4M3 output's rel-L2 against the bf16
+    forward's.  One JSON line."""
+    import dataclasses
+    from block_sparse_attention_12_b200 import abi, build
+    build.build()
+    torch.cuda.set_device(0)
+    w = inputs.WORKLOADS[args.workload]
+    if args.heads:
+        w = dataclasses.replace(w, H=args.heads)
+    Q, K, V = inputs.make_qkv(w, device="cuda:0")
+    cfg = abi.Config(kv_block=w.kv_block, budget=w.budget, n_clusters=w.n_clusters,
+                     kmeans_iters=w.kmeans_iters, seed=w.seed)
+    stream = torch.cuda.current_stream()
+    plan = abi.plan(Q, K, cfg)
+    O, lse = abi.forward(Q, K, V, plan, cfg)
+    Q8, qs = abi.quantize_e4m3(Q, 128)
+    K8, ks = abi.quantize_e4m3(K, w.kv_block)
+    O8, lse8 = abi.forward_e4m3(Q8, qs, K8, ks, V, plan, cfg)
+    abi.check()
+    n_it = max(3, args.steps)
+    t_bf = timed(lambda: abi.forward(Q, K, V, plan, cfg, O=O, lse=lse), n_it, stream)
+    t_q = timed(lambda: (abi.quantize_e4m3(Q, 128, codes=Q8, scales=qs),
+                         abi.quantize_e4m3(K, w.kv_block, codes=K8, scales=ks)), n_it, stream)
+    t_8 = timed(lambda: abi.forward_e4m3(Q8, qs, K8, ks, V, plan, cfg, O=O8, lse=lse8), n_it, stream)
+    abi.check()
+    fl = abi.executed_flops(plan, tuple(Q.shape))
+    d = O8.float() - O.float()
+    print(json.dumps({
+        "e4m3_forward": w.name, "heads": w.H, "tokens": w.N,
+        "bf16_forward_ms": t_bf, "bf16_forward_tflops": fl / (t_bf / 1e3) / 1e12,
+        "e4m3_forward_ms": t_8, "e4m3_forward_tflops": fl / (t_8 / 1e3) / 1e12,
+        "quantize_q_and_k_ms": t_q,
+        "e4m3_vs_bf16_output_rel_l2": float(d.norm() / O.float().norm()),
+        "note": "QK^T in E4M3 (Q scaled per 128-query block, K per KV block); P and V bf16",
+    }), flush=True)
+
+
 def run_gather_bench(args):
     """Cycles per 128-key tile to gather the 32 selected 4-row blocks of K and
     V (64 KB) into a 3-stage shared-memory ring, for each copy method and
@@ -479,6 +522,9 @@ def main():
         return
     if args.mma_bench:
         run_mma_bench(args)
+        return
+    if args.e4m3:
+        run_e4m3(args)
         return
     if args.sweep:
         run_sweep(args)

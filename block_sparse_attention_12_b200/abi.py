@@ -27,6 +27,7 @@ EXPORTED = [
     "abattn_plan_workspace_size", "abattn_score_workspace_size", "abattn_meanpool",
     "abattn_kmeans", "abattn_score", "abattn_plan_from_scores", "abattn_plan_from_pi",
     "abattn_plan", "abattn_forward", "abattn_dense_forward", "abattn_plan_noalloc",
+    "abattn_quantize_e4m3", "abattn_forward_e4m3",
 ]
 
 
@@ -93,6 +94,8 @@ def lib():
         L.abattn_forward.argtypes = [VP, VP, VP, P_D, P_P, VP, VP, VP, ctypes.c_int64, VP, VP, VP]
         L.abattn_dense_forward.argtypes = [VP, VP, VP, P_D, ctypes.c_float, VP, VP, VP]
         L.abattn_plan_noalloc.argtypes = [VP, VP, P_D, P_P, VP, VP, VP, ctypes.c_int64, VP]
+        L.abattn_quantize_e4m3.argtypes = [VP, P_D, ctypes.c_int, VP, VP, VP]
+        L.abattn_forward_e4m3.argtypes = [VP, VP, VP, VP, VP, P_D, P_P, VP, VP, VP, ctypes.c_int64, VP, VP, VP]
         for name in EXPORTED:
             if name not in ("abattn_version", "abattn_strerror"):
                 getattr(L, name).restype = ctypes.c_int
@@ -290,6 +293,42 @@ def forward(Q, K, V, plan: Plan, cfg: Config | None = None, O=None, lse=None, wa
     _ok(lib().abattn_forward(_ptr(Q), _ptr(K), _ptr(V), ctypes.byref(dims_of(Q)), ctypes.byref(cfg.params()),
                              _ptr(plan.counts), _ptr(plan.idx), _ptr(plan.pi_sel), plan.cap, _ptr(O), _ptr(lse),
                              _stream(stream)), "abattn_forward")
+    return O, lse
+
+
+def quantize_e4m3(X, rows_per_block: int, codes=None, scales=None, stream=None):
+    """bf16 [B, H, N, 128] -> (E4M3 codes uint8 [B, H, N, 128], scales fp32
+    [B, H, ceil(N / rows_per_block)]), one scale per block of rows (128 rows for
+    Q, the plan's kv_block for K)."""
+    _check_qkv(X)
+    B, H, N, d = X.shape
+    if codes is None:
+        codes = torch.empty(B, H, N, d, dtype=torch.uint8, device=X.device)
+    if scales is None:
+        scales = torch.empty(B, H, -(-N // rows_per_block), dtype=torch.float32, device=X.device)
+    _ok(lib().abattn_quantize_e4m3(_ptr(X), ctypes.byref(dims_of(X)), int(rows_per_block), _ptr(codes),
+                                   _ptr(scales), _stream(stream)), "abattn_quantize_e4m3")
+    return codes, scales
+
+
+def forward_e4m3(Q8, q_scales, K8, k_scales, V, plan: Plan, cfg: Config | None = None, O=None, lse=None,
+                 want_lse=True, stream=None):
+    """The gathered sparse forward with QK^T in E4M3 (Q8, K8 and their scales
+    from quantize_e4m3: 128 rows per block for Q, the plan's kv_block for K);
+    V bf16 [B, H, N, 128]."""
+    _check_qkv(V)
+    for t in (Q8, K8):
+        if t.dtype != torch.uint8 or t.shape != V.shape or not t.is_contiguous():
+            raise ValueError("E4M3 codes must be contiguous uint8 tensors shaped like V")
+    cfg = cfg or Config(kv_block=plan.kv_block)
+    if O is None:
+        O = torch.empty_like(V)
+    if lse is None and want_lse:
+        lse = torch.empty(V.shape[:3], dtype=torch.float32, device=V.device)
+    _ok(lib().abattn_forward_e4m3(_ptr(Q8), _ptr(q_scales), _ptr(K8), _ptr(k_scales), _ptr(V),
+                                  ctypes.byref(dims_of(V)), ctypes.byref(cfg.params()), _ptr(plan.counts),
+                                  _ptr(plan.idx), _ptr(plan.pi_sel), plan.cap, _ptr(O), _ptr(lse),
+                                  _stream(stream)), "abattn_forward_e4m3")
     return O, lse
 
 

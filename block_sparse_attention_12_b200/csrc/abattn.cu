@@ -11,6 +11,7 @@
 #include "common.cuh"
 #include "forward.cuh"
 #include "planner.cuh"
+#include "quant.cuh"
 #include "selector.cuh"
 
 using namespace abattn;
@@ -92,6 +93,21 @@ int make_map_rows(CUtensorMap *m, const void *base, int64_t d, int64_t rows, int
 // Q, K, V [B][H][N][d] as {d, N, B*H}.
 int make_map(CUtensorMap *m, const void *base, const abattn_dims *d, int box_rows) {
     return make_map_rows(m, base, d->d, d->N, d->B * d->H, box_rows);
+}
+
+// E4M3 codes [B][H][N][128] as a byte tensor {128, N, B*H}; box {128, 128, 1}
+// (one 128-byte row per query), 128-byte swizzle, zero fill.
+int make_map_e4m3(CUtensorMap *m, const void *base, const abattn_dims *d) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return ABATTN_ERR_DEVICE;
+    cuuint64_t dims[3] = {128u, cuuint64_t(d->N), cuuint64_t(d->B * d->H)};
+    cuuint64_t strides[2] = {128u, cuuint64_t(d->N * 128)};
+    cuuint32_t box[3] = {128u, 128u, 1u};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? ABATTN_OK : ABATTN_ERR_CUDA;
 }
 
 int check_device() {
@@ -299,12 +315,52 @@ int run_forward(bool dense, const void *Q, const void *K, const void *V, const a
     fp.box_rows = box;
     fp.nkvb = int(cdiv(d->N, fp.kb));
     fp.scale_log2 = resolve_scale(scale, d->d) * 1.4426950408889634f;
+    fp.q_scale = nullptr;
+    fp.k_scale = nullptr;
     const int64_t rows = d->B * d->H * fp.nqb;
     // every kv block starts at a multiple of 4 keys (kb is 4, 8, ..., 128), so
     // with N % 4 == 0 each 4-key group of a tile is entirely valid or entirely past N
     const bool grouped = (d->N % 4) == 0;
     if (d->d == 128) return launch_fwd_hd<128>(dense, grouped, mQ, mK, mV, fp, rows, st);
     return launch_fwd_hd<64>(dense, grouped, mQ, mK, mV, fp, rows, st);
+}
+
+// The E4M3 forward: sparse, grouped (N % 4 == 0), d = 128.
+int run_forward_e4m3(const void *Q8, const float *q_scale, const void *K8, const float *k_scale, const void *V,
+                     const abattn_dims *d, int kb, float scale, const int32_t *counts, const int32_t *idx,
+                     const float *pi_sel, int64_t cap, void *O, float *lse, cudaStream_t st) {
+    int rc = check_device();
+    if (rc) return rc;
+    CUtensorMap mQ, mV;
+    if ((rc = make_map_e4m3(&mQ, Q8, d)) || (rc = make_map(&mV, V, d, 32))) return rc;
+    FwdParams fp;
+    fp.K = static_cast<const __nv_bfloat16 *>(K8);  // E4M3 codes, read as bytes
+    fp.V = static_cast<const __nv_bfloat16 *>(V);
+    fp.counts = counts;
+    fp.idx = idx;
+    fp.pi_sel = pi_sel;
+    fp.cap = cap;
+    fp.O = static_cast<__nv_bfloat16 *>(O);
+    fp.lse = lse;
+    fp.N = int(d->N);
+    fp.nqb = int(cdiv(d->N, 128));
+    fp.kb = kb;
+    fp.box_rows = 32;
+    fp.nkvb = int(cdiv(d->N, kb));
+    fp.scale_log2 = resolve_scale(scale, d->d) * 1.4426950408889634f;
+    fp.q_scale = q_scale;
+    fp.k_scale = k_scale;
+    const int64_t rows = d->B * d->H * fp.nqb;
+    constexpr int smem = FwdLayout<128, true>::ALLOC;
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(fwd_kernel<128, false, true, true>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return cuda_status(e);
+        attr = true;
+    }
+    fwd_kernel<128, false, true, true><<<unsigned(rows), FWD_THREADS, smem, st>>>(mQ, mQ, mV, fp);
+    return launch_status();
 }
 
 int check_plan_shape(const abattn_dims *d, const abattn_params *p) {
@@ -498,6 +554,41 @@ int abattn_forward(const void *Q, const void *K, const void *V, const abattn_dim
     if (cap < 1 || cap > cdiv(dims->N, p->kv_block)) return ABATTN_ERR_SHAPE;
     return run_forward(false, Q, K, V, dims, p->kv_block, p->scale, counts, idx, pi_sel, cap, O, lse,
                        static_cast<cudaStream_t>(stream));
+}
+
+int abattn_quantize_e4m3(const void *X, const abattn_dims *dims, int rows_per_block, void *codes, float *scales,
+                         void *stream) {
+    int rc = check_dims(dims);
+    if (rc) return rc;
+    if (dims->d != 128) return ABATTN_ERR_SHAPE;
+    if (rows_per_block < 1 || rows_per_block > 128 || (rows_per_block & (rows_per_block - 1)))
+        return ABATTN_ERR_PARAM;
+    if (X == nullptr || codes == nullptr || scales == nullptr) return ABATTN_ERR_NULL;
+    if (!aligned16(X) || !aligned16(codes)) return ABATTN_ERR_ALIGN;
+    if ((rc = check_device())) return rc;
+    const int64_t batches = dims->B * dims->H;
+    if (batches > 65535) return ABATTN_ERR_SHAPE;
+    const dim3 grid(unsigned(cdiv(dims->N, QZ_THREADS)), unsigned(batches));
+    quant_e4m3_kernel<<<grid, QZ_THREADS, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const __nv_bfloat16 *>(X), dims->N, rows_per_block, cdiv(dims->N, rows_per_block),
+        static_cast<uint8_t *>(codes), scales);
+    return launch_status();
+}
+
+int abattn_forward_e4m3(const void *Q8, const float *q_scales, const void *K8, const float *k_scales,
+                        const void *V, const abattn_dims *dims, const abattn_params *p, const int32_t *counts,
+                        const int32_t *idx, const float *pi_sel, int64_t cap, void *O, float *lse, void *stream) {
+    int rc = check_dims(dims);
+    if (rc) return rc;
+    if ((rc = check_params(p, false))) return rc;
+    if (dims->d != 128 || dims->N % 4 != 0) return ABATTN_ERR_SHAPE;
+    if (Q8 == nullptr || q_scales == nullptr || K8 == nullptr || k_scales == nullptr || V == nullptr ||
+        O == nullptr || counts == nullptr || idx == nullptr || pi_sel == nullptr)
+        return ABATTN_ERR_NULL;
+    if (!aligned16(Q8) || !aligned16(K8) || !aligned16(V) || !aligned16(O)) return ABATTN_ERR_ALIGN;
+    if (cap < 1 || cap > cdiv(dims->N, p->kv_block)) return ABATTN_ERR_SHAPE;
+    return run_forward_e4m3(Q8, q_scales, K8, k_scales, V, dims, p->kv_block, p->scale, counts, idx, pi_sel, cap,
+                            O, lse, static_cast<cudaStream_t>(stream));
 }
 
 int abattn_dense_forward(const void *Q, const void *K, const void *V, const abattn_dims *dims, float scale,

@@ -220,6 +220,19 @@ __device__ __forceinline__ void umma_ss_lo(uint32_t d_tmem, uint32_t a_lo, uint3
         "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(kSdescHi), "r"(accumulate)
         : "memory");
 }
+// D[tmem] (+)= A[smem] * B[smem], kind::f8f6f4 (K = 32 one-byte elements per
+// MMA), descriptors as for umma_ss_lo.
+__device__ __forceinline__ void umma_f8_ss_lo(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t idesc,
+                                              uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "mov.b64 da, {%1, %4};\n\t"
+        "mov.b64 db, {%2, %4};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], da, db, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(kSdescHi), "r"(accumulate)
+        : "memory");
+}
 __device__ __forceinline__ void umma_ts_lo(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t idesc,
                                            uint32_t accumulate) {
     asm volatile(
@@ -248,6 +261,16 @@ __host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, int a_mn, i
            | (1u << 10)                       // B format: bf16
            | (uint32_t(a_mn) << 15)           // A major
            | (uint32_t(b_mn) << 16)           // B major
+           | (uint32_t(N >> 3) << 17)         // N / 8
+           | (uint32_t(M >> 4) << 24);        // M / 16
+}
+
+// Instruction descriptor of a kind::f8f6f4 MMA with E4M3 A and B (type code 0),
+// fp32 accumulator, both operands K-major.
+__host__ __device__ constexpr uint32_t make_idesc_e4m3(int M, int N) {
+    return (1u << 4)                          // D format: f32
+           | (0u << 7)                        // A format: E4M3
+           | (0u << 10)                       // B format: E4M3
            | (uint32_t(N >> 3) << 17)         // N / 8
            | (uint32_t(M >> 4) << 24);        // M / 16
 }

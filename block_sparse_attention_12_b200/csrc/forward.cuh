@@ -86,21 +86,34 @@ struct FwdParams {
     int box_rows;  // dense kernel: rows per K/V TMA box (32)
     int nkvb;
     float scale_log2;
+    // E4M3 forward only: the scale of each 128-query block [rows] and of each
+    // KV block [B*H][nkvb]; K then holds E4M3 codes [B*H][N][128]
+    const float *q_scale;
+    const float *k_scale;
 };
 
-template <int HD>
+// FP8: Q and K as E4M3 codes (d = 128: one 128-byte row per query or key, so
+// a 16 KB tile), V bf16; the smaller tiles leave room for a fourth stage.
+template <int HD, bool FP8 = false>
 struct FwdLayout {
     static constexpr int HALVES = HD / 64;
     static constexpr int TILE = HALVES * 16384;  // 128 rows x HD bf16, per 64-col half 16 KB
+    static constexpr int NS = FP8 ? 4 : FWD_NS;  // K/V stages
+    static constexpr int QT = FP8 ? 16384 : TILE;
+    static constexpr int KT = FP8 ? 16384 : TILE;
+    static constexpr int VT = TILE;
     static constexpr int Q_OFF = 0;
-    static constexpr int K_OFF = Q_OFF + TILE;
-    static constexpr int V_OFF = K_OFF + FWD_NS * TILE;
+    static constexpr int K_OFF = Q_OFF + QT;
+    static constexpr int V_OFF = K_OFF + NS * KT;
     // per-key bias [NS][128] (N % 4 != 0) or per-group bias [NS][32]: one
     // kernel uses one of the two, so they share the area
-    static constexpr int BIAS_OFF = V_OFF + FWD_NS * TILE;
+    static constexpr int BIAS_OFF = V_OFF + NS * VT;
     static constexpr int GBIAS_OFF = BIAS_OFF;
-    static constexpr int BAR_OFF = BIAS_OFF + FWD_NS * 128 * 4;
-    static constexpr int NBARS = 1 + 2 * FWD_NS + 8;
+    // FP8: each 4-key group's logit multiplier (query-block scale x KV-block
+    // scale x softmax scale) [NS][32]
+    static constexpr int MUL_OFF = BIAS_OFF + NS * 128 * 4;
+    static constexpr int BAR_OFF = MUL_OFF + (FP8 ? NS * 32 * 4 : 0);
+    static constexpr int NBARS = 1 + 2 * NS + 8;
     // (m, l) of both softmax warpgroups, [2][2][128] floats, exchanged in the
     // epilogue through the first K stage: by then every QK^T MMA has completed
     // and every K load has landed
@@ -113,11 +126,18 @@ struct FwdLayout {
 // GROUPED (N % 4 == 0): every 4-key group of a tile shares one bias, since
 // block boundaries are multiples of 4 keys and so is N; the softmax then adds
 // the bias once per group.  Otherwise the bias is kept per key.
-template <int HD, bool DENSE, bool GROUPED>
+//
+// FP8 (sparse, grouped, d = 128 only): Q and K are E4M3 codes with one scale per
+// 128-query block and per KV block (the VC-Attention pages' 8-bit attention on
+// B200); QK^T runs as E4M3 MMAs and each group's logits are multiplied by its
+// block's scales; P and V stay bf16.
+template <int HD, bool DENSE, bool GROUPED, bool FP8 = false>
 __global__ void __launch_bounds__(FWD_THREADS, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
-    using L = FwdLayout<HD>;
+    static_assert(!FP8 || (!DENSE && GROUPED && HD == 128), "E4M3 forward: sparse, grouped, d = 128");
+    using L = FwdLayout<HD, FP8>;
+    constexpr int NS = L::NS;
     extern __shared__ uint8_t fwd_smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(fwd_smem_raw) + 1023) & ~uintptr_t(1023));
@@ -126,11 +146,12 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
     uint8_t *sV = smem + L::V_OFF;
     float *sBias = reinterpret_cast<float *>(smem + L::BIAS_OFF);
     float *sGBias = reinterpret_cast<float *>(smem + L::GBIAS_OFF);
+    float *sMul = reinterpret_cast<float *>(smem + L::MUL_OFF);  // FP8 only
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::BAR_OFF);
     uint64_t *q_full = bars;
     uint64_t *kv_full = bars + 1;
-    uint64_t *kv_empty = bars + 1 + FWD_NS;
-    uint64_t *s_full = bars + 1 + 2 * FWD_NS;  // [2]
+    uint64_t *kv_empty = bars + 1 + NS;
+    uint64_t *s_full = bars + 1 + 2 * NS;  // [2]
     uint64_t *p_full = s_full + 2;              // [2 warpgroups][2 key halves]
     uint64_t *pv_done = p_full + 4;             // [2]
     float *xch = reinterpret_cast<float *>(smem + L::XCH_OFF);
@@ -154,7 +175,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
-        for (int s = 0; s < FWD_NS; ++s) {
+        for (int s = 0; s < NS; ++s) {
             // dense: one expect_tx arrival per producer warp (TMA bytes);
             // sparse: one cp.async completion arrival per producer thread plus
             // one release arrival per warp for the biases
@@ -191,9 +212,13 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         int issued = 0;
         if (T > 0) {
             if (lane == 0 && pw == 0) {
-                mbar_arrive_expect_tx(q_full, 128 * HD * 2);
+                mbar_arrive_expect_tx(q_full, L::QT);
+                if constexpr (FP8) {
+                    tma_load_3d(sQ, &tmQ, q_full, 0, q0, bh);  // 128 rows x 128 E4M3 codes
+                } else {
 #pragma unroll
-                for (int h = 0; h < L::HALVES; ++h) tma_load_3d(sQ + h * 16384, &tmQ, q_full, h * 64, q0, bh);
+                    for (int h = 0; h < L::HALVES; ++h) tma_load_3d(sQ + h * 16384, &tmQ, q_full, h * 64, q0, bh);
+                }
             }
             const int32_t *ridx = DENSE ? nullptr : p.idx + int64_t(row) * p.cap;
             const float *rpi = DENSE ? nullptr : p.pi_sel + int64_t(row) * p.cap;
@@ -210,8 +235,8 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                 const int nown = nunits > pw ? (nunits - pw + FWD_PRODUCERS - 1) / FWD_PRODUCERS : 0;
                 const uint32_t tx_bytes = uint32_t(nown) * R * HD * 2 * 2;
                 for (int t = 0; t < T; ++t) {
-                    const int s = t % FWD_NS;
-                    if (t >= FWD_NS && !mbar_wait(&kv_empty[s], ((t / FWD_NS) - 1) & 1, abort_flag)) break;
+                    const int s = t % NS;
+                    if (t >= NS && !mbar_wait(&kv_empty[s], ((t / NS) - 1) & 1, abort_flag)) break;
                     if (owner) {
                         const int key0 = t * kb + ro;
                         if constexpr (GROUPED) {
@@ -224,8 +249,8 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                         __syncwarp(__activemask());
                         if (lane == 0) mbar_arrive_expect_tx(&kv_full[s], tx_bytes);
                         __syncwarp(__activemask());
-                        uint8_t *dK = sK + s * L::TILE + unit * R * 128;
-                        uint8_t *dV = sV + s * L::TILE + unit * R * 128;
+                        uint8_t *dK = sK + s * L::KT + unit * R * 128;
+                        uint8_t *dV = sV + s * L::VT + unit * R * 128;
 #pragma unroll
                         for (int h = 0; h < L::HALVES; ++h) {
                             tma_load_3d(dK + h * 16384, &tmK, &kv_full[s], h * 64, key0, bh);
@@ -284,21 +309,31 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                 float cur_pi, nxt_pi;
                 fetch(0, cur_blk, cur_pi);
                 fetch(1, nxt_blk, nxt_pi);
+                // FP8: the KV-block scale of the entries of tiles t (cur) and
+                // t+1 (nxt, loaded at the top of iteration t), and the query
+                // block's scale times the softmax scale
+                auto fetch_ks = [&](int blk) -> float {
+                    return (owner && blk >= 0 && blk < p.nkvb) ? __ldg(p.k_scale + int64_t(bh) * p.nkvb + blk) : 0.f;
+                };
+                const float qmul = FP8 ? __ldg(p.q_scale + row) * p.scale_log2 : 0.f;
+                float cur_ks = FP8 ? fetch_ks(cur_blk) : 0.f, nxt_ks = 0.f;
                 for (int t = 0; t < T; ++t) {
-                    const int s = t % FWD_NS;
+                    const int s = t % NS;
                     int x_blk;
                     float x_pi;
                     fetch(t + 2, x_blk, x_pi);
-                    if (t >= FWD_NS && !mbar_wait(&kv_empty[s], ((t / FWD_NS) - 1) & 1, abort_flag)) break;
-                    // this lane's quad: block, first key and bias
+                    if constexpr (FP8) nxt_ks = fetch_ks(nxt_blk);
+                    if (t >= NS && !mbar_wait(&kv_empty[s], ((t / NS) - 1) & 1, abort_flag)) break;
+                    // this lane's quad: block, first key, bias and (FP8) multiplier
                     int key0 = 0;
-                    float b = -INFINITY;
+                    float b = -INFINITY, mq = 0.f;
                     if (owner) {
                         int blk = fill_blk;  // padding slot: loaded, weighted zero
                         if (t * spt + sl < cnt) {
                             if (cur_blk >= 0 && cur_blk < p.nkvb && cur_pi > 0.f) {
                                 blk = cur_blk;
                                 b = -log2f(cur_pi);
+                                if constexpr (FP8) mq = qmul * cur_ks;
                             } else if (ro == 0) {
                                 raise_error(kErrBounds);
                             }
@@ -312,14 +347,23 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                         const int key = k0 + r;
                         const bool valid = key < p.N;  // rows past N (ragged last block) read as zero
                         const int srow = q * 4 + r;
-                        const uint32_t soff = uint32_t(s * L::TILE + srow * 128 + ((c ^ (srow & 7)) << 4));
+                        const uint32_t roff = uint32_t(srow * 128 + ((c ^ (srow & 7)) << 4));
                         const int64_t goff = int64_t(valid ? key : 0) * HD + c * 8;
+                        if constexpr (FP8) {
+                            // the K row is 128 E4M3 codes: one 16-byte chunk per lane
+                            const uint8_t *K8bh = reinterpret_cast<const uint8_t *>(p.K) + int64_t(bh) * p.N * 128;
+                            cp_async16(sK + s * L::KT + roff, K8bh + int64_t(valid ? key : 0) * 128 + c * 16, valid);
+                        }
 #pragma unroll
                         for (int h = 0; h < L::HALVES; ++h) {
-                            cp_async16(sK + soff + h * 16384, Kbh + goff + h * 64, valid);
-                            cp_async16(sV + soff + h * 16384, Vbh + goff + h * 64, valid);
+                            if constexpr (!FP8) cp_async16(sK + s * L::KT + roff + h * 16384, Kbh + goff + h * 64, valid);
+                            cp_async16(sV + s * L::VT + roff + h * 16384, Vbh + goff + h * 64, valid);
                         }
                         if constexpr (GROUPED) {
+                            if constexpr (FP8) {
+                                const float mj = __shfl_sync(0xffffffffu, mq, j);
+                                if (lane == 0) sMul[s * 32 + q] = mj;
+                            }
                             if (lane == 0) sGBias[s * 32 + q] = k0 < p.N ? bj : -INFINITY;
                         } else {
                             if (c == 0) sBias[s * 128 + q * 4 + r] = valid ? bj : -INFINITY;
@@ -332,6 +376,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                     cur_pi = nxt_pi;
                     nxt_blk = x_blk;
                     nxt_pi = x_pi;
+                    cur_ks = nxt_ks;
                     ++issued;
                 }
                 cp_async_wait_all();
@@ -341,8 +386,8 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                 if (lane == 0) {
                     if (pw == 0) mbar_drain(q_full, 0);
                     if (DENSE)
-                        for (int t = issued - FWD_NS < 0 ? 0 : issued - FWD_NS; t < issued; ++t)
-                            mbar_drain(&kv_full[t % FWD_NS], (t / FWD_NS) & 1);
+                        for (int t = issued - NS < 0 ? 0 : issued - NS; t < issued; ++t)
+                            mbar_drain(&kv_full[t % NS], (t / NS) & 1);
                 }
             }
         }
@@ -358,18 +403,26 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
             // V as an MN-major operand LBO 16384 (its second 64-column half)
             const uint32_t q_lo = sdesc_lo(aQ, 16), k_lo = sdesc_lo(aK, 16), v_lo = sdesc_lo(aV, 16384);
             auto issue_qk = [&](int t) -> bool {
-                const int s = t % FWD_NS, sb = t & 1;
-                if (!mbar_wait(&kv_full[s], (t / FWD_NS) & 1, abort_flag)) return false;
+                const int s = t % NS, sb = t & 1;
+                if (!mbar_wait(&kv_full[s], (t / NS) & 1, abort_flag)) return false;
                 // the sparse tile was written by cp.async (generic proxy): order
                 // those writes, observed through the barrier, before the MMAs'
                 // async-proxy reads
                 if (!DENSE) fence_proxy_async_smem();
                 tc_fence_after();
-                const uint32_t kb_lo = k_lo + uint32_t(s) * (L::TILE >> 4);
+                const uint32_t kb_lo = k_lo + uint32_t(s) * (L::KT >> 4);
+                if constexpr (FP8) {
+                    // E4M3: 32 codes (32 bytes) of the 128-byte rows per MMA
+                    constexpr uint32_t idesc_qk8 = make_idesc_e4m3(128, 128);
 #pragma unroll
-                for (int k = 0; k < HD / 16; ++k) {
-                    const uint32_t off = ((k >> 2) * 16384 + (k & 3) * 32) >> 4;
-                    umma_ss_lo(tmem + sb * 128, q_lo + off, kb_lo + off, idesc_qk, k > 0 ? 1u : 0u);
+                    for (int k = 0; k < 4; ++k)
+                        umma_f8_ss_lo(tmem + sb * 128, q_lo + k * 2, kb_lo + k * 2, idesc_qk8, k > 0 ? 1u : 0u);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < HD / 16; ++k) {
+                        const uint32_t off = ((k >> 2) * 16384 + (k & 3) * 32) >> 4;
+                        umma_ss_lo(tmem + sb * 128, q_lo + off, kb_lo + off, idesc_qk, k > 0 ? 1u : 0u);
+                    }
                 }
                 umma_commit(&s_full[sb]);
                 return true;
@@ -378,8 +431,8 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
             for (int t = 0; ok && t < T; ++t) {
                 if (t + 1 < T && !issue_qk(t + 1)) break;
                 const int g = t & 1;  // softmax warpgroup / S buffer / O accumulator of this tile
-                const int s = t % FWD_NS;
-                const uint32_t vb_lo = v_lo + uint32_t(s) * (L::TILE >> 4);
+                const int s = t % NS;
+                const uint32_t vb_lo = v_lo + uint32_t(s) * (L::VT >> 4);
                 const uint32_t pbase = tmem + g * 128;
                 const uint32_t acc0 = t >= 2 ? 1u : 0u;
                 if constexpr (DENSE) {
@@ -424,9 +477,9 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         bool ok = true;
         int ntiles = 0;
         for (int t = g; t < T; t += 2, ++ntiles) {
-            const int s = t % FWD_NS;
+            const int s = t % NS;
             if (!mbar_wait(&s_full[g], (t >> 1) & 1, abort_flag) ||
-                !mbar_wait(&kv_full[s], (t / FWD_NS) & 1, abort_flag)) {
+                !mbar_wait(&kv_full[s], (t / NS) & 1, abort_flag)) {
                 ok = false;
                 break;
             }
@@ -436,6 +489,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
             for (int c = 0; c < 4; ++c) tmem_ld32(t_S + c * 32, x[c]);
             tmem_wait_ld();
             const float *gbias = sGBias + s * 32;
+            const float *gmul = sMul + s * 32;  // FP8: each group's logit multiplier
             const float *bias = sBias + s * 128;
             const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
             float2 rs01 = make_float2(0.f, 0.f), rs23 = make_float2(0.f, 0.f);
@@ -481,8 +535,14 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                         float gm[4];
 #pragma unroll
                         for (int j = 0; j < 4; ++j) gm[j] = gmax(q0 + j);
-                        const float2 v01 = __ffma2_rn(make_float2(gm[0], gm[1]), sc2, make_float2(g4.x, g4.y));
-                        const float2 v23 = __ffma2_rn(make_float2(gm[2], gm[3]), sc2, make_float2(g4.z, g4.w));
+                        float2 m01 = sc2, m23 = sc2;  // (FP8: the groups' multipliers, all positive)
+                        if constexpr (FP8) {
+                            const float4 u4 = *reinterpret_cast<const float4 *>(gmul + q0);
+                            m01 = make_float2(u4.x, u4.y);
+                            m23 = make_float2(u4.z, u4.w);
+                        }
+                        const float2 v01 = __ffma2_rn(make_float2(gm[0], gm[1]), m01, make_float2(g4.x, g4.y));
+                        const float2 v23 = __ffma2_rn(make_float2(gm[2], gm[3]), m23, make_float2(g4.z, g4.w));
                         mt0 = fmax3(mt0, v01.x, v01.y);
                         mt1 = fmax3(mt1, v23.x, v23.y);
                     } else {
@@ -510,15 +570,21 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
             auto exp_pass = [&](float m_ref, int qa) {
 #pragma unroll
                 for (int q0 = qa; q0 < qa + 16; q0 += 4) {
-                    float4 g4;
+                    float4 g4, u4;
                     if constexpr (GROUPED) g4 = *reinterpret_cast<const float4 *>(gbias + q0);
+                    if constexpr (FP8) u4 = *reinterpret_cast<const float4 *>(gmul + q0);
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const int q = q0 + j;
                         if constexpr (GROUPED) {
                             const float gb = j == 0 ? g4.x : j == 1 ? g4.y : j == 2 ? g4.z : g4.w;
                             const float2 off = make_float2(gb - m_ref, gb - m_ref);
-                            exp_group(q, xa(q), xb(q), sc2, off, off);
+                            float2 mul = sc2;
+                            if constexpr (FP8) {
+                                const float mu = j == 0 ? u4.x : j == 1 ? u4.y : j == 2 ? u4.z : u4.w;
+                                mul = make_float2(mu, mu);
+                            }
+                            exp_group(q, xa(q), xb(q), mul, off, off);
                         } else {
                             const float2 neg_m = make_float2(-m_ref, -m_ref);
                             exp_group(q, xa(q), xb(q), make_float2(1.f, 1.f), neg_m, neg_m);

@@ -11,6 +11,11 @@
  *       SIP and fine-grained-kernel paragraphs; the last one also says the
  *       sampling plan is rebuilt once every four denoising steps while the
  *       attention runs every step, hence the plan / forward split below.
+ *  [P3], [P4] "Nunchux AI VC-Attention speeds up video DiT inference 3.58x"
+ *       (dothoosh news, Persian) and "Nunchux AI ra mat VC-Attention"
+ *       (aihot, Vietnamese): 8-bit (E4M3) attention on B200, the source of
+ *       the optional E4M3 forward below; a different method, whose
+ *       quantisation is not part of AB-Attention.
  *
  * Conventions for every entry point
  *  - Tensors are device pointers, caller-allocated and caller-owned; the
@@ -160,6 +165,34 @@ int abattn_plan(const void *Q, const void *K, const abattn_dims *dims, const aba
 int abattn_forward(const void *Q, const void *K, const void *V, const abattn_dims *dims,
                    const abattn_params *p, const int32_t *counts, const int32_t *idx,
                    const float *pi_sel, int64_t cap, void *O, float *lse, void *stream);
+
+/* E4M3 block quantisation for the 8-bit forward ([P3], [P4], B200 results:
+ * 8-bit attention on Blackwell).  X bf16 [B][H][N][d] with d = 128 ->
+ * codes [B][H][N][d] (one byte each) and scales fp32 [B][H][ceil(N / rpb)].
+ * Each block of rows_per_block consecutive rows (a power of two from 1 to
+ * 128; the last block of a head may be short) gets scale = amax / 448, amax
+ * the largest |x| in the block (1 for a block of zeros), and each element the
+ * E4M3 code of fp32(x * fp32(448 / amax)), rounded to nearest even and
+ * saturated at +-448 (E4M3: 1 sign, 4 exponent bits with bias 7, 3 mantissa
+ * bits).  Use 128 rows per block for Q (one scale per query block) and
+ * p->kv_block for K (one scale per KV block).  Errors: ABATTN_ERR_SHAPE for
+ * d != 128, ABATTN_ERR_PARAM for another block size; nothing is launched
+ * after a host-side error. */
+int abattn_quantize_e4m3(const void *X, const abattn_dims *dims, int rows_per_block, void *codes,
+                         float *scales, void *stream);
+
+/* The gathered block-sparse forward with QK^T in E4M3: as abattn_forward,
+ * with Q and K given as abattn_quantize_e4m3 codes and scales (Q with 128
+ * rows per block, K with p->kv_block), so that each logit is
+ *   scale * q_scale[query block] * k_scale[KV block] * (Q8 . K8)
+ *     + ln(1/pi_j)
+ * from E4M3 tensor-core products with fp32 accumulation; P and V stay bf16,
+ * as in abattn_forward.  Requires d = 128 and N % 4 == 0 (ABATTN_ERR_SHAPE
+ * otherwise).  O bf16 [B][H][N][d]; lse fp32 [B][H][N] (nullable). */
+int abattn_forward_e4m3(const void *Q8, const float *q_scales, const void *K8, const float *k_scales,
+                        const void *V, const abattn_dims *dims, const abattn_params *p,
+                        const int32_t *counts, const int32_t *idx, const float *pi_sel, int64_t cap,
+                        void *O, float *lse, void *stream);
 
 /* Dense softmax attention ([P1] bottleneck section: 3D full attention), the
  * full-budget reference, same kernel design over all keys.  scale 0 means

@@ -182,3 +182,35 @@ def test_dense_rows_against_oracle(layer):
         Og = O[0, 0, q0:q0 + 16].float().cpu().numpy().astype(np.float64)
         check_forward(w, Og, Oo, Ao, f"dense rows {q0}..{q0 + 15} (h {h})")
         np.testing.assert_allclose(lse[0, 0, q0:q0 + 16].cpu().numpy(), lo, atol=2e-3, rtol=1e-4)
+
+
+def test_e4m3_forward_rows_against_oracle(layer):
+    """The E4M3 forward on the layer's plan, for the sampled rows: against the
+    oracle on the dequantised Q and K (same bound as the bf16 forward), and its
+    rel-L2 against the oracle on the bf16 inputs printed."""
+    w, plan, cfg = layer["w"], layer["plan"], layer["cfg"]
+    if w.d != 128:
+        pytest.skip("the E4M3 forward takes d = 128")
+    Q8, qs = abi.quantize_e4m3(layer["Q"], 128)
+    K8, ks = abi.quantize_e4m3(layer["K"], w.kv_block)
+    O8, lse8 = abi.forward_e4m3(Q8, qs, K8, ks, layer["V"], plan, cfg)
+    abi.check()
+    scale = 1 / math.sqrt(w.d)
+    for b, h, qb in layer["rows"][:3]:
+        _, _, v = layer["data"][h]
+        q0 = qb * 128
+        M = min(128, w.N - q0)
+        qd = oracle.dequantize_e4m3_rows(Q8[b, h].cpu().numpy(), qs[b, h].cpu().numpy(), 128)[q0:q0 + M]
+        kd = oracle.dequantize_e4m3_rows(K8[b, h].cpu().numpy(), ks[b, h].cpu().numpy(), w.kv_block)
+        n = int(plan.counts[b, h, qb])
+        idx = plan.idx[b, h, qb, :n].cpu().numpy()
+        ps = plan.pi_sel[b, h, qb, :n].cpu().numpy()
+        Oo, lo_ = oracle.sparse_block(qd, kd, v, w.kv_block, idx, ps, scale)
+        Ao, _ = oracle.sparse_block(qd, kd, np.abs(v), w.kv_block, idx, ps, scale)
+        Og = O8[b, h, q0:q0 + M].float().cpu().numpy().astype(np.float64)
+        check_forward(w, Og, Oo, Ao, f"E4M3 row (h {h}, qb {qb})")
+        np.testing.assert_allclose(lse8[b, h, q0:q0 + M].cpu().numpy(), lo_, atol=2e-3, rtol=1e-4)
+        q, k, _ = layer["data"][h]
+        Ox, _ = oracle.sparse_block(q[q0:q0 + M], k, v, w.kv_block, idx, ps, scale)
+        print(f"{w.name} E4M3 row (h {h}, qb {qb}) vs the bf16 inputs: rel-L2 "
+              f"{np.linalg.norm(Og - Ox) / np.linalg.norm(Ox):.3e}")
