@@ -50,7 +50,7 @@ def parse():
     ap.add_argument("--workload", default="wan14b-720p", choices=sorted(inputs.WORKLOADS))
     ap.add_argument("--heads", type=int, default=0,
                     help="run only this many heads of the layer (small cases for ncu captures)")
-    ap.add_argument("--e2e-steps", type=int, default=6)
+    ap.add_argument("--e2e-steps", type=int, default=16)
     ap.add_argument("--dense-iters", type=int, default=3)
     ap.add_argument("--cpu-rows", type=int, default=64)
     ap.add_argument("--cpu-rows-one-core", type=int, default=12)
@@ -713,10 +713,31 @@ def main():
             dist.barrier()
         e2e_ms = multigpu.max_over_ranks(e2e_run(args.e2e_steps), Q.device)
         abi.check()
+        h2d = 3 * Q.numel() * Q.element_size()
+
+        # the host link alone: one step's uploads with nothing else running
+        # (best of three), the bound that the pipelined steps approach
+        def upload_ms():
+            ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            ea.record(s_in)
+            with torch.cuda.stream(s_in):
+                for t_d, t_h in zip(dev[0][:3], (Qh, Kh, Vh)):
+                    t_d.copy_(t_h, non_blocking=True)
+            eb.record(s_in)
+            torch.cuda.synchronize()
+            return ea.elapsed_time(eb)
+
+        up_ms = min(upload_ms() for _ in range(3))
         e2e = {"value": multigpu.job_throughput(exec_fl, e2e_ms, world) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
-               "h2d_bytes_per_step": 3 * Q.numel() * Q.element_size(),
+               "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": O.numel() * O.element_size(),
-               "pipelining": "upload of step k+1 and download of step k-1 overlap step k (3 streams)"}
+               "steps": args.e2e_steps,
+               "pipelining": "upload of step k+1 and download of step k-1 overlap step k (3 streams); "
+                             "the time includes the pipeline's fill and drain",
+               "h2d_gbs_alone": h2d / (up_ms * 1e6),
+               "link_bound_ms": up_ms,
+               "link_frac": up_ms / e2e_ms}
         del Qh, Kh, Vh, Oh, dev
 
     cpu = None
