@@ -91,11 +91,13 @@ __global__ void split_rows_kernel(const float *__restrict__ src, int64_t nblk, i
 // One CTA (128 threads, one warpgroup) per q-block; both Lloyd steps run on
 // the tensor cores, with the block's queries staged once by TMA in the
 // 128-byte-swizzled K-major layout:
-//   assignment: D_a[query][c] = q . c for 16 centroid slots (8 used) as
-//               Q [128 x d] times (C_hi + C_lo)^T, two bf16 MMA groups into
-//               one fp32 TMEM accumulator (the queries are exactly bf16, the
-//               fp32 centroids split into a bf16 pair hi + lo); thread i
-//               (TMEM lane i) then takes argmin_c |c|^2 - 2 q.c (the same
+//   assignment: D_a[query][c] = q . c for 16 centroid slots (8 used); the
+//               queries are exactly bf16 and the fp32 centroids are split
+//               into a bf16 pair hi + lo, stacked as the 32 rows of one B
+//               operand (rows 0..15 hi, 16..31 lo), so each k-step is one
+//               N = 32 MMA and columns c and 16 + c of the fp32 TMEM
+//               accumulator hold q . c_hi and q . c_lo; thread i (TMEM lane
+//               i) adds the two and takes argmin_c |c|^2 - 2 q.c (the same
 //               argmin as |q - c|^2), ties to the lower index;
 //   update:     D_u[k][c] = sum of dimension k over cluster c's members as
 //               Q^T [d x 128] times a one-hot [128 x 16] assignment matrix;
@@ -106,17 +108,20 @@ __global__ void split_rows_kernel(const float *__restrict__ src, int64_t nblk, i
 // iterations early with the same result.  For d = 64 the tile's second
 // 64-column half is zero, so the update still has M = 128 rows.  Thread k
 // keeps the fp32 centroids of dimension k in registers, and the one-hot
-// operand shares its tile with the centroids' lo part (the assignment has
-// read that before the one-hot is written, the update has read the one-hot
-// before the new centroids are), so five CTAs fit an SM.
+// operand takes the rows of the centroids' lo part (the assignment has read
+// those before the one-hot is written, the update has read the one-hot before
+// the new centroids are), so five CTAs fit an SM.  MMAs of N = 16 or 32 cost
+// close to a fixed time each, so the stacked hi/lo operand halves the
+// assignment's share of the tensor pipe (8 MMAs a k-sweep instead of 16).
 constexpr int KM_THREADS = 128;
 
 struct KmLayout {
     static constexpr int Q_OFF = 0;          // [2 halves][128 rows][128 B]
-    static constexpr int CHI_OFF = 32768;    // [2 halves][16 rows][128 B]
-    static constexpr int CLO_OFF = 36864;    // the same, or the one-hot [2 query halves][16 rows][128 B]
-    static constexpr int OH_OFF = CLO_OFF;
-    static constexpr int CN_OFF = CLO_OFF + 4096;        // |c|^2 [8], partials [4][8]
+    static constexpr int C_HALF = 4096;      // bytes between the 64-column halves of the centroid operand
+    static constexpr int CHI_OFF = 32768;    // [2 halves][32 rows][128 B]: rows 0..15 hi, 16..31 lo
+    static constexpr int CLO_OFF = CHI_OFF + 2048;  // rows 16..31 of each half
+    static constexpr int OH_OFF = CLO_OFF;   // or the one-hot [2 query halves][16 rows][128 B] in those rows
+    static constexpr int CN_OFF = CHI_OFF + 2 * C_HALF;  // |c|^2 [8], partials [4][8]
     static constexpr int INT_OFF = CN_OFF + 40 * 4;      // lab[128], cnt[8], wcnt[4][8]
     static constexpr int BAR_OFF = INT_OFF + (128 + 8 + 32) * 4;  // q_bar, mma_bar
     static constexpr int MISC_OFF = BAR_OFF + 16;         // tmem slot
@@ -158,7 +163,7 @@ __global__ void __launch_bounds__(KM_THREADS, 5) kmeans_kernel(
     const int M = int(N - q0 < 128 ? N - q0 : 128);
 
     if (wid == 0) {
-        tmem_alloc(tmem_slot, 32);  // D_a: columns [0, 16), D_u: [16, 32)
+        tmem_alloc(tmem_slot, 64);  // D_a: columns [0, 32), D_u: [32, 48)
         tmem_relinquish();
     }
     if (tid == 0) {
@@ -171,7 +176,7 @@ __global__ void __launch_bounds__(KM_THREADS, 5) kmeans_kernel(
     // and, for d = 64, the tile's second half
     {
         uint4 *z = reinterpret_cast<uint4 *>(smem + L::CHI_OFF);
-        for (int e = tid; e < (2 * 4096) / 16; e += KM_THREADS) z[e] = make_uint4(0, 0, 0, 0);
+        for (int e = tid; e < (2 * L::C_HALF) / 16; e += KM_THREADS) z[e] = make_uint4(0, 0, 0, 0);
         if (D == 64) {
             uint4 *zq = reinterpret_cast<uint4 *>(sQ + 16384);
             for (int e = tid; e < 16384 / 16; e += KM_THREADS) zq[e] = make_uint4(0, 0, 0, 0);
@@ -202,7 +207,7 @@ __global__ void __launch_bounds__(KM_THREADS, 5) kmeans_kernel(
         cs[c] = v;
         __nv_bfloat16 hi, lo;
         split_bf16(v, hi, lo);
-        const uint32_t o = sw128_off(c, k, 2048);
+        const uint32_t o = sw128_off(c, k, L::C_HALF);
         *reinterpret_cast<__nv_bfloat16 *>(sChi + o) = hi;
         *reinterpret_cast<__nv_bfloat16 *>(sClo + o) = lo;
         return v * v;
@@ -231,7 +236,7 @@ __global__ void __launch_bounds__(KM_THREADS, 5) kmeans_kernel(
     }
     if (tid < 8) cnt_s[tid] = 0;
 
-    constexpr uint32_t idesc_a = make_idesc_bf16(128, 16, 0, 0);  // Q . C^T
+    constexpr uint32_t idesc_a = make_idesc_bf16(128, 32, 0, 0);  // Q . [C_hi; C_lo]^T
     constexpr uint32_t idesc_u = make_idesc_bf16(128, 16, 1, 0);  // Q^T . onehot, A MN-major
     uint32_t phase = 0;
     for (int it = 0; ok && it < iters; ++it) {
@@ -239,31 +244,28 @@ __global__ void __launch_bounds__(KM_THREADS, 5) kmeans_kernel(
         if (tid == 0) {
             tc_fence_after();
             const uint32_t q_lo = sdesc_lo(smem_u32(sQ), 16);
-            const uint32_t hi_lo = sdesc_lo(smem_u32(sChi), 16), lo_lo = sdesc_lo(smem_u32(sClo), 16);
+            const uint32_t c_lo = sdesc_lo(smem_u32(sChi), 16);
 #pragma unroll
             for (int k = 0; k < D / 16; ++k) {
-                const uint32_t qo = ((k >> 2) * 16384 + (k & 3) * 32) >> 4, co = ((k >> 2) * 2048 + (k & 3) * 32) >> 4;
-                umma_ss_lo(tmem, q_lo + qo, hi_lo + co, idesc_a, k > 0 ? 1u : 0u);
-            }
-#pragma unroll
-            for (int k = 0; k < D / 16; ++k) {
-                const uint32_t qo = ((k >> 2) * 16384 + (k & 3) * 32) >> 4, co = ((k >> 2) * 2048 + (k & 3) * 32) >> 4;
-                umma_ss_lo(tmem, q_lo + qo, lo_lo + co, idesc_a, 1u);
+                const uint32_t qo = ((k >> 2) * 16384 + (k & 3) * 32) >> 4,
+                               co = ((k >> 2) * L::C_HALF + (k & 3) * 32) >> 4;
+                umma_ss_lo(tmem, q_lo + qo, c_lo + co, idesc_a, k > 0 ? 1u : 0u);
             }
             umma_commit(mma_bar);
         }
         ok = mbar_wait(mma_bar, phase, abort_flag);
         phase ^= 1;
         tc_fence_after();
-        uint32_t a16[16];
-        tmem_ld16(t_lane, a16);
+        uint32_t a32[32];
+        tmem_ld32(t_lane, a32);
         tmem_wait_ld();
         int best = 0;
         {
-            float bd = fmaf(-2.f, __uint_as_float(a16[0]), cn[0]);
+            // q . c = (q . c_hi) + (q . c_lo), columns c and 16 + c
+            float bd = fmaf(-2.f, __uint_as_float(a32[0]) + __uint_as_float(a32[16]), cn[0]);
 #pragma unroll
             for (int c = 1; c < 8; ++c) {
-                const float v = fmaf(-2.f, __uint_as_float(a16[c]), cn[c]);
+                const float v = fmaf(-2.f, __uint_as_float(a32[c]) + __uint_as_float(a32[16 + c]), cn[c]);
                 if (c < nc && v < bd) { bd = v; best = c; }
             }
         }
@@ -280,7 +282,7 @@ __global__ void __launch_bounds__(KM_THREADS, 5) kmeans_kernel(
             const unsigned m = __ballot_sync(0xffffffffu, tid < M && best == c);
             if (lane == 0) wcnt[wid * 8 + c] = __popc(m);
             const __nv_bfloat16 one = __float2bfloat16(tid < M && best == c ? 1.f : 0.f);
-            *reinterpret_cast<__nv_bfloat16 *>(sOH + sw128_off(c, tid, 2048)) = one;
+            *reinterpret_cast<__nv_bfloat16 *>(sOH + sw128_off(c, tid, L::C_HALF)) = one;
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -291,8 +293,8 @@ __global__ void __launch_bounds__(KM_THREADS, 5) kmeans_kernel(
             const uint32_t qt_lo = sdesc_lo(smem_u32(sQ), 16384), oh_lo = sdesc_lo(smem_u32(sOH), 16);
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
-                const uint32_t oo = ((k >> 2) * 2048 + (k & 3) * 32) >> 4;
-                umma_ss_lo(tmem + 16, qt_lo + k * (2048 >> 4), oh_lo + oo, idesc_u, k > 0 ? 1u : 0u);
+                const uint32_t oo = ((k >> 2) * L::C_HALF + (k & 3) * 32) >> 4;
+                umma_ss_lo(tmem + 32, qt_lo + k * (2048 >> 4), oh_lo + oo, idesc_u, k > 0 ? 1u : 0u);
             }
             umma_commit(mma_bar);
         }
@@ -300,7 +302,7 @@ __global__ void __launch_bounds__(KM_THREADS, 5) kmeans_kernel(
         phase ^= 1;
         tc_fence_after();
         uint32_t s16[16];
-        tmem_ld16(t_lane + 16, s16);
+        tmem_ld16(t_lane + 32, s16);
         tmem_wait_ld();
         ok = __syncthreads_and(ok) != 0;  // (also publishes cnt_s)
         if (!ok) break;
@@ -335,7 +337,7 @@ __global__ void __launch_bounds__(KM_THREADS, 5) kmeans_kernel(
     __syncthreads();
     if (wid == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, 32);
+        tmem_dealloc(tmem, 64);
     }
 }
 
