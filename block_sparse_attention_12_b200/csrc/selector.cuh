@@ -110,9 +110,9 @@ __global__ void split_rows_kernel(const float *__restrict__ src, int64_t nblk, i
 // keeps the fp32 centroids of dimension k in registers, and the one-hot
 // operand takes the rows of the centroids' lo part (the assignment has read
 // those before the one-hot is written, the update has read the one-hot before
-// the new centroids are), so five CTAs fit an SM.  MMAs of N = 16 or 32 cost
-// close to a fixed time each, so the stacked hi/lo operand halves the
-// assignment's share of the tensor pipe (8 MMAs a k-sweep instead of 16).
+// the new centroids are), so five CTAs fit an SM.  The kernel is bound by the
+// latency of its two dependent MMA round trips per iteration; the stacked
+// hi/lo operand halves the first one (8 MMAs a k-sweep instead of 16).
 constexpr int KM_THREADS = 128;
 
 struct KmLayout {
