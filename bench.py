@@ -635,9 +635,9 @@ def main():
         "meanpool": {"bound": "hbm", "unit": "GB/s", "peak": P["hbm"],
                      "work": BH * w.N * w.d * 2 + BH * nkvb * w.d * 4,
                      "traffic": traffic_for("meanpool", BH * nkvb)},
-        # k-means (both Lloyd steps on tcgen05, 16-column accumulators) is bound by
-        # the latency of its dependent iterations; its roofline is its one read of
-        # the queries (and the centroid, weight and label writes)
+        # k-means (both Lloyd steps on tcgen05) is bound by the latency of its
+        # dependent iterations; its roofline is its one read of the queries (and
+        # the centroid, weight and label writes)
         "kmeans": {"bound": "hbm", "unit": "GB/s", "peak": P["hbm"],
                    "work": rows * (128 * w.d * 2 + w.n_clusters * w.d * 4 + w.n_clusters * 4 + 128 * 4),
                    "traffic": traffic_for("kmeans", rows)},
